@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""KDA on B200: prefill tokens/s at B=1, H=16, T=65536 and decode state GB/s.
+
+One step = one ``kda_chunk_fwd`` call over a B=1, H=16, T=65536, d=128 bf16
+sequence with a random fp32 initial state (plan + segment summary + combine +
+output kernels).  The decode figure is measured in the same run on the
+B=256, H=32 decode workload (512 MiB fp32 state updated in place).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs its
+own independent sequence (weak scaling, no collective on the data path) and
+the step time is the max over ranks.  ``--impl reference`` times the fp64
+oracle (the plain CPU statement of the method) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+T_PREFILL, H_PREFILL, D = 65536, 16, 128
+BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + D * 4 + 4   # q,k,v + o (bf16), g (fp32), beta
+FLOP_PER_TOKEN_HEAD = 6 * D * D + 3 * 64 * D + 64 * 64  # the pages' per-head count, C = 64
+
+
+def metric_name():
+    try:
+        with open(os.path.join(ROOT, "BASELINE.json")) as f:
+            return json.load(f)["metric"]
+    except Exception:
+        return "KDA prefill tokens/s (H=16,T=64K) + decode state GB/s, % of B200 roofline"
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", str(self.gpu),
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_oracle_sample(T_s: int, H_s: int, seed: int = 77):
+    """Time the fp64 oracle on H_s heads x T_s tokens of the prefill workload."""
+    import numpy as np
+    import oracle
+    import synth
+    inp = synth.op_inputs(**{**synth.prefill_sweep(T_PREFILL), "T": T_s, "H": H_s, "seed": seed})
+    f = lambda t: t.double().numpy()  # noqa: E731
+    args = [f(inp[n]) for n in ("q", "k", "v", "g", "beta")]
+    s0 = f(inp["s0"])
+    t0 = time.perf_counter()
+    oracle.kda_recurrent(*args, s0=s0)
+    dt = time.perf_counter() - t0
+    return dt, oracle.num_threads()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    T_s, H_s = 2048, H_PREFILL
+    times = []
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        dt, cores = cpu_oracle_sample(T_s, H_s, seed=100 + i)
+        if i >= args.warmup:
+            times.append(dt)
+    t = statistics.mean(times)
+    value = T_s / t  # tokens/s with all 16 heads of each token
+    line = {
+        "metric": metric_name(), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"KDA prefill B=1 H=16 d=128, oracle sample of {T_s} tokens x {H_s} heads per step",
+                   "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{T_s} tokens x {H_s} heads of the B=1,H=16,T=65536 prefill, per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import gated_delta_rule_123_b200 as kda
+    import synth
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    T = args.T
+    cfg = dict(synth.prefill_sweep(T))
+    cfg["seed"] += 1000 * rank
+    inp = synth.op_inputs(**cfg, device=dev)
+    q, k, v, g, beta, s0 = (inp[n] for n in ("q", "k", "v", "g", "beta", "s0"))
+    o = torch.empty_like(q)
+    fs = torch.empty_like(s0)
+    wsz = kda.chunk_fwd_workspace_bytes(1, T, H_PREFILL)
+    ws = torch.empty(wsz, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.chunk_fwd(q, k, v, g, beta, initial_state=s0, out=o, final_state=fs, workspace=ws)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_w = time.perf_counter()
+    n_w = 0
+    while n_w < args.warmup or time.perf_counter() - t_w < args.warmup_seconds:
+        step()
+        n_w += 1
+        if n_w % 10 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+
+    # timed region: K steps, per-kernel trace events on the launching stream
+    traces = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        kda.set_trace_events(traces[i])
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    kda.set_trace_events(None)
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms)
+    out_ms = statistics.mean(tr[3].elapsed_time(tr[4]) for tr in traces)
+    sum_ms = statistics.mean(tr[1].elapsed_time(tr[2]) for tr in traces)
+    comb_ms = statistics.mean(tr[2].elapsed_time(tr[3]) for tr in traces)
+    plan_ms = statistics.mean(tr[0].elapsed_time(tr[1]) for tr in traces)
+    assert kda.device_status() == 0
+    value = world * T / (ms / 1e3)
+
+    # roofline of the dominant kernel (the output pass): algorithmic bytes per launch / its time
+    alg_bytes = BYTES_PER_TOKEN_HEAD * T * H_PREFILL
+    achieved = alg_bytes / (out_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None, "kernel": "chunk_kernel<output>",
+                "peak_kind": peak_kind,
+                "step_frac": alg_bytes / (ms / 1e3) / 1e9 / hbm_peak,
+                "kernel_ms": {"plan": plan_ms, "summary": sum_ms, "combine": comb_ms, "output": out_ms},
+                "tensor_tflops_step": FLOP_PER_TOKEN_HEAD * T * H_PREFILL / (ms / 1e3) / 1e12,
+                "tensor_peak": tc_peak}
+
+    if args.prefill_only:
+        if rank == 0:
+            print(json.dumps({"metric": metric_name(), "value": value, "unit": "tokens/s", "ms_per_step": ms,
+                              "config": {"workload": f"KDA prefill B=1 H=16 T={T} (prefill only)"},
+                              "roofline": roofline}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # decode: B=256, H=32, state updated in place (inputs cycled from a pool of 8 seeded steps)
+    dcfg = synth.DECODE_B256
+    B, H = dcfg["B"], dcfg["H"]
+    S = synth.decode_state(B, H, seed=dcfg["seed"] + rank, device=dev)
+    pool = [synth.decode_step_inputs(B, H, i, seed=dcfg["seed"], device=dev) for i in range(8)]
+    od = torch.empty_like(pool[0]["q"])
+
+    def dstep(i):
+        p = pool[i % 8]
+        kda.decode_step(p["q"], p["k"], p["v"], p["g"], p["beta"], S, out=od)
+
+    for i in range(5):
+        dstep(i)
+    n_dec = 200
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(n_dec):
+        dstep(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    dec_us = max_over_ranks(start.elapsed_time(end) / n_dec * 1e3)
+    dec_bytes = 2 * B * H * D * D * 4 + B * H * (4 * D * 2 + D * 4 + 4)
+    dec_gbs = dec_bytes / (dec_us / 1e6) / 1e9
+    assert kda.device_status() == 0
+
+    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hfs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    dq, dk, dv, dg, db, ds0 = (torch.empty_like(t) for t in (q, k, v, g, beta, s0))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hs0))
+    d2h = ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size()
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (ds0, hs0)):
+            d_.copy_(h_, non_blocking=True)
+        kda.chunk_fwd(dq, dk, dv, dg, db, initial_state=ds0, out=o, final_state=fs, workspace=ws)
+        ho.copy_(o, non_blocking=True)
+        hfs.copy_(fs, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    start.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(start.elapsed_time(end) / e2e_steps)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        T_s, H_s = 4096, H_PREFILL
+        dt, cores = cpu_oracle_sample(T_s, H_s)
+        cpu = {"value": T_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{T_s} tokens x {H_s} heads of the B=1,H=16,T=65536 prefill ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": metric_name(), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"KDA prefill B=1 H=16 T={T} d=128 bf16, fp32 g/beta/state "
+                                   "(one independent sequence per GPU)",
+                       "l2": "inputs larger than L2 (1.6 GB per step)", "parallelism": f"replicas x{world}"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "decode": {"workload": "B=256 H=32 d=128, fp32 state in place", "us_per_step": dec_us,
+                       "gbs": dec_gbs, "peak_gbs": hbm_peak, "frac": dec_gbs / hbm_peak,
+                       "tokens_per_s": world * B / (dec_us / 1e6)},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=T_PREFILL, help="prefill length (profiling runs use a smaller one)")
+    ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and the CPU baseline")
+    ap.add_argument("--warmup-seconds", type=float, default=1.5, help="minimum warm-up time (clock sampling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

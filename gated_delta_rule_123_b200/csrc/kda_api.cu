@@ -1,0 +1,168 @@
+// extern "C" entry points of libkda: host-side argument validation, then
+// launches on the caller's stream.  Declared and documented in include/kda.h.
+#include <stdio.h>
+#include <string.h>
+
+#include "kda_common.cuh"
+
+namespace kda {
+
+int launch_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       float* state, void* o, int B, int H, int dtype, float scale, int l2norm, cudaStream_t stream);
+int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
+                     int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
+                     const char** why);
+size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
+size_t layer_workspace_bytes(int total_tokens, int d_model, int H, int rank, int num_seqs);
+int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int num_seqs, int total_tokens,
+                     const float* init, float* fin, void* y, void* ws, size_t ws_bytes, cudaStream_t stream,
+                     const char** why);
+
+static thread_local char t_last_error[256] = "";
+thread_local cudaEvent_t* g_trace_events = nullptr;
+
+static int fail(int code, const char* msg) {
+    snprintf(t_last_error, sizeof(t_last_error), "%s", msg ? msg : "");
+    return code;
+}
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_status_string(int s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+int kda_head_dim(void) { return kD; }
+
+const char* kda_last_error(void) { return t_last_error; }
+
+int kda_set_trace_events(void* events, int n_events) {
+    if (events && n_events < 5) return fail(KDA_ERR_INVALID_ARG, "need 5 events");
+    g_trace_events = static_cast<cudaEvent_t*>(events);
+    return KDA_OK;
+}
+
+int kda_device_status(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int val = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&val, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return fail(KDA_ERR_CUDA, cudaGetErrorString(cudaGetLastError()));
+    if (val != 0) {
+        cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+        cudaStreamSynchronize(s);
+        char msg[64];
+        snprintf(msg, sizeof(msg), "device wait gave up (site mask 0x%x)", val);
+        return fail(KDA_ERR_TIMEOUT, msg);
+    }
+    return KDA_OK;
+}
+
+size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk) {
+    if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;
+    return chunk_workspace_bytes(B, T, H, num_seqs, dtype, l2norm_qk);
+}
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens, int num_seqs,
+                  int B, int T, int H, int dtype, float scale, int l2norm_qk, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
+    if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if (cu_seqlens) {
+        if (B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1");
+        if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires num_seqs >= 1");
+    } else if (num_seqs != 0) {
+        return fail(KDA_ERR_INVALID_ARG, "num_seqs must be 0 for dense input");
+    }
+    const long long N = cu_seqlens ? num_seqs : B;
+    if ((long long)(cu_seqlens ? 1 : B) * T * H * kD >= (1ll << 31))
+        return fail(KDA_ERR_UNSUPPORTED, "more than 2^31 elements per token tensor");
+    if ((long long)T * H * kD == 0 || N == 0 || H == 0) {
+        // nothing to compute except the state pass-through
+        if (final_state && N * H > 0) {
+            const size_t bytes = size_t(N) * H * kD * kD * sizeof(float);
+            cudaError_t e = initial_state
+                                ? (initial_state == final_state
+                                       ? cudaSuccess
+                                       : cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice,
+                                                         static_cast<cudaStream_t>(stream)))
+                                : cudaMemsetAsync(final_state, 0, bytes, static_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess) return fail(KDA_ERR_CUDA, cudaGetErrorString(e));
+        }
+        return KDA_OK;
+    }
+    if (!q || !k || !v || !g || !beta || !o) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o) ||
+        (initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (o == q || o == k || o == v) return fail(KDA_ERR_INVALID_ARG, "o must not alias q, k or v");
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char* why = "";
+    const int rc = launch_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H,
+                                    dtype, scale, l2norm_qk, workspace, workspace_bytes,
+                                    static_cast<cudaStream_t>(stream), &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,
+                    void* o, int B, int H, int dtype, float scale, int l2norm_qk, void* stream) {
+    t_last_error[0] = 0;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
+    if (B < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if ((long long)B * H == 0) return KDA_OK;
+    if ((long long)B * H >= (1ll << 31)) return fail(KDA_ERR_UNSUPPORTED, "too many heads");
+    if (!q || !k || !v || !g || !beta || !state || !o) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o))
+        return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    const int rc = launch_decode_step(q, k, v, g, beta, state, o, B, H, dtype, scale, l2norm_qk,
+                                      static_cast<cudaStream_t>(stream));
+    return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
+}
+
+size_t kda_layer_fwd_workspace(int total_tokens, int d_model, int H, int rank, int num_seqs) {
+    if (total_tokens < 0 || d_model <= 0 || H <= 0 || rank <= 0 || num_seqs < 1) return 0;
+    return layer_workspace_bytes(total_tokens, d_model, H, rank, num_seqs);
+}
+
+int kda_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu_seqlens, int num_seqs,
+                  int total_tokens, const float* initial_state, float* final_state, void* y, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    if (!w) return fail(KDA_ERR_INVALID_ARG, "NULL weights");
+    if (w->d_model <= 0 || w->H <= 0 || w->rank <= 0 || total_tokens < 0 || num_seqs < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes");
+    if (w->d_model % 8 || w->rank % 8) return fail(KDA_ERR_UNSUPPORTED, "d_model and rank must be multiples of 8");
+    if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is required");
+    if (total_tokens == 0) return KDA_OK;
+    if (!x || !y || !w->W_in || !w->W_aup || !w->W_gup || !w->conv_w || !w->norm_w || !w->W_o)
+        return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(y) || !aligned16(w->W_in) || !aligned16(w->W_aup) || !aligned16(w->W_gup) ||
+        !aligned16(w->W_o) || (initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char* why = "";
+    const int rc = launch_layer_fwd(x, w, cu_seqlens, num_seqs, total_tokens, initial_state, final_state, y, workspace,
+                                    workspace_bytes, static_cast<cudaStream_t>(stream), &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
+}
+
+}  // extern "C"

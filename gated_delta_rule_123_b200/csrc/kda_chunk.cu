@@ -1,0 +1,899 @@
+// KDA chunkwise prefill on sm_100a: TMA-fed tcgen05 tiles, fp32 state in TMEM.
+//
+// The method ("Kimi Linear: An Expressive, Efficient Attention Architecture",
+// section "Chunkwise Algorithm"; the news rewrite "Kimi Linear", section on the
+// hardware-efficient chunkwise algorithm): split every sequence into chunks of
+// C = 64 tokens; inside a chunk unroll the per-channel decay and the rank-1
+// corrections (WY representation), invert the unit lower-triangular system by
+// forward substitution (UT transform), and carry only the 128x128 state from
+// chunk to chunk.  Per chunk, with b the in-chunk cumulative log decay
+// (gamma^{i->j} = prod_{k=i+1}^{j} alpha^k, the corrected definition from the
+// section "Mathematical Rigor"):
+//     A[r,i] = beta_r sum_c k_rc k_ic exp(b_rc - b_ic)      (i < r)
+//     P[r,i] =        sum_c q_rc k_ic exp(b_rc - b_ic)      (i <= r)
+//     T = (I + A)^{-1}
+//     W = T diag(beta) (K (.) e^b),   U = T diag(beta) V     (one T for both:
+//                                      the a = b = sqrt(beta) k binding)
+//     U~ = U - W S,   O = (Q (.) e^b) S + P U~,
+//     S' = Diag(e^{b_C}) S + (K (.) e^{b_C - b})^T U~.
+//
+// B200 design (what differs from the pages' GPU design):
+//  * Everything is computed transposed so that every tensor-core tile has
+//    M = 128 (one TMEM lane per key or value channel): S^T lives in TMEM as the
+//    fp32 accumulator (lane = value channel, column = key channel) for the
+//    whole sequence segment; one thread per lane owns its row.
+//  * The gated operands are formed ONCE per chunk from a per-channel reference
+//    point m_c = (b_0c + b_63c)/2: Kp = K (.) e^{b-m}, Qp = Q (.) e^{b-m},
+//    Km = K (.) e^{m-b}.  Then A = diag(beta) Kp Km^T and P = Qp Km^T (one
+//    stacked M=128 MMA), W S = (T beta Kp) (Diag(e^m) S), Q e^b S = Qp
+//    (Diag(e^m) S), and the state update becomes
+//    S' = Diag(e^{b_C - m}) [Diag(e^m) S + Km^T U~]: the Diag factors are
+//    per-lane scalings folded into the one TMEM pass per chunk that also
+//    writes the bf16 copy of S used as the MMA operand.  Every exponent is
+//    bounded by half the chunk's decay range (checked per chunk); chunks whose
+//    range exceeds kRangeMax take an exact fallback (A, P on CUDA cores with
+//    one exp per term; the other products with m = 0 / b_C references, whose
+//    factors are all <= 1).
+//  * Long sequences with few (sequence, head) pairs are cut into segments so
+//    that ~one CTA per SM has work: a summary pass computes each segment's
+//    affine map S_end = X S_start + N (X carried like a second state with
+//    U = 0), a short combine pass chains the maps, and the output pass runs
+//    every segment from its true start state.  Only the state crosses chunks.
+#include <cub/block/block_scan.cuh>
+
+#include "kda_common.cuh"
+
+namespace kda {
+
+extern thread_local cudaEvent_t* g_trace_events;
+
+struct SegItem {
+    int seq;        // sequence index n
+    int tok_begin;  // first token of this segment (packed index)
+    int tok_end;    // one past its last token
+    int g;          // segment index inside the sequence
+    int G;          // number of segments of the sequence
+    int first;      // item index of segment 0 of the sequence
+    int pad0, pad1;
+};
+
+constexpr float kRangeMax = 64.f;   // max in-chunk decay range (nats) for the factored path
+constexpr float kGateFloor = -1e4f; // log-gates below this are treated as this
+
+// Shared-memory plan (bytes from a 1024-aligned base).  Tiles are bf16 with
+// 128-byte swizzled rows unless noted.
+constexpr uint32_t OFF_Q = 0;         // [64 tok][128 c]  (two 64-column boxes, TMA)
+constexpr uint32_t OFF_K = 16384;     // [64 tok][128 c]  (TMA)
+constexpr uint32_t OFF_V = 32768;     // [64 tok][128 v]  (TMA; MN-major A of U^T)
+constexpr uint32_t OFF_G = 49152;     // fp32 [64 tok][128 c] (TMA, no swizzle)
+constexpr uint32_t OFF_KP = 81920;    // [128 c][64 tok]  Kp
+constexpr uint32_t OFF_QP = 98304;    // [128 c][64 tok]  Qp (must follow Kp by 16 KB)
+constexpr uint32_t OFF_KM = 114688;   // [128 c][64 tok]  Km
+constexpr uint32_t OFF_TB = 131072;   // [64 r][64 i]     T diag(beta)
+constexpr uint32_t OFF_P = 139264;    // [64 r][64 i]     P (lower incl. diagonal)
+constexpr uint32_t OFF_WN = 147456;   // [128 k][64 tok]  -W^T  (also fp32 A scratch)
+constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S^T (operand copy)
+constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T (also fp32 T scratch)
+constexpr uint32_t OFF_MISC = 212992;
+constexpr uint32_t MISC_BYTES = 7 * 1024;
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+// Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
+
+// TMEM columns (512 allocated): S^T | [A;P] | W^T | U^T | O^T (or U_X^T) | X^T
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_U = 256, TM_O = 320, TM_X = 384;
+
+struct ChunkArgs {
+    const float* beta;
+    const float* init_state;
+    float* final_state;
+    void* o;
+    const SegItem* items;
+    const int* n_items;
+    float* segN;
+    float* segX;
+    const float* segS;
+    int H;
+    float scale;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// kSummary = true : segment summary (zero start state, identity X, no output).
+// kSummary = false: output pass from the segment's true start state.
+template <bool kSummary, typename OutT>
+__global__ void __launch_bounds__(256, 1)
+    chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                 const ChunkArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    const uint32_t sbase = smem_u32(sm);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
+    if (item_id >= *p.n_items) return;
+    const SegItem it = p.items[item_id];
+    if (kSummary && it.g == it.G - 1) return;  // the last segment's map is never needed
+
+    float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC);  // [64]
+    float* sPreOp = sBeta + 64;                                // [128]
+    float* sPreAcc = sPreOp + 128;                             // [128]
+    float* sPost = sPreAcc + 128;                              // [2][128]
+    float* sCarry = sPost + 256;                               // [256]
+    float* sX = sCarry + 256;                                  // [768]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 768);    // qkg, v, mma
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+    float* sA = reinterpret_cast<float*>(sm + OFF_WN);  // fp32 [64][64] scratch
+    float* sT = reinterpret_cast<float*>(sm + OFF_UT);  // fp32 [64][64] scratch
+
+    if (warp == 0) {
+        tmem_alloc(sTmem, 512);
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbar_init();
+    }
+    if (tid == 64) {
+        if (!kSummary) prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_g);
+    }
+    if (tid < 128) sPost[128 + tid] = 1.f;  // the "previous chunk" of chunk 0 scales by 1
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *sTmem;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const int vrow = quad * 32 + lane;  // TMEM lane owned by this thread
+
+    const int t_begin = it.tok_begin, t_end = it.tok_end;
+    const int nchunks = (t_end - t_begin + kC - 1) / kC;
+
+    auto issue_qkg = [&](int c) {
+        const int t0 = t_begin + c * kC;
+        mbar_arrive_expect_tx(&bars[0], kSummary ? 49152u : 65536u);
+        if (!kSummary) {
+            tma_load_3d(sm + OFF_Q, &tm_q, &bars[0], 0, h, t0);
+            tma_load_3d(sm + OFF_Q + 8192, &tm_q, &bars[0], 64, h, t0);
+        }
+        tma_load_3d(sm + OFF_K, &tm_k, &bars[0], 0, h, t0);
+        tma_load_3d(sm + OFF_K + 8192, &tm_k, &bars[0], 64, h, t0);
+        tma_load_3d(sm + OFF_G, &tm_g, &bars[0], 0, h, t0);
+    };
+    auto issue_v = [&](int c) {
+        const int t0 = t_begin + c * kC;
+        mbar_arrive_expect_tx(&bars[1], 16384u);
+        tma_load_3d(sm + OFF_V, &tm_v, &bars[1], 0, h, t0);
+        tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[1], 64, h, t0);
+    };
+    bool pend_qkg = false, pend_v = false;  // meaningful in thread 0 only
+    if (tid == 0 && nchunks > 0) {
+        issue_qkg(0);
+        issue_v(0);
+        pend_qkg = pend_v = true;
+    }
+
+    // ---- start state into TMEM: S^T (lane = v, column = k); X^T = I for the summary.
+    {
+        const float* src = nullptr;
+        if (!kSummary) {
+            // A segmented sequence takes every start state (segment 0's too) from
+            // the combine pass, so final_state may alias initial_state.
+            if (it.G == 1)
+                src = p.init_state ? p.init_state + (size_t(it.seq) * H + h) * (kD * kD) : nullptr;
+            else
+                src = p.segS + (size_t(item_id) * H + h) * (kD * kD);
+        }
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            float buf[16];
+            const int k0 = half * 64 + cb * 16;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) buf[j] = src ? src[size_t(k0 + j) * kD + vrow] : 0.f;
+            tmem_st16(tbase + TM_S + lane_off + k0, buf);
+            if (kSummary) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) buf[j] = (k0 + j == vrow) ? 1.f : 0.f;
+                tmem_st16(tbase + TM_X + lane_off + k0, buf);
+            }
+        }
+        tmem_wait_st();
+    }
+
+    uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
+    bool aborted = false;
+    const uint32_t id_ap = idesc_bf16(128, 64, 1, 1);   // [Kp;Qp] (MN) x Km (MN)
+    const uint32_t id_w = idesc_bf16(128, 64, 0, 0);    // Kp^T (K) x (T beta)^T (K)
+    const uint32_t id_u = idesc_bf16(128, 64, 1, 0);    // V^T (MN) x (T beta)^T (K)
+    const uint32_t id_so = idesc_bf16(128, 64, 0, 1);   // S^T (K) x {-W^T, Qp} (MN)
+    const uint32_t id_po = idesc_bf16(128, 64, 0, 0);   // U~^T (K) x P^T (K)
+    const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // U~^T (K) x Km (K)
+    const uint32_t XT0 = kSummary ? OFF_Q : 0, XT1 = kSummary ? OFF_QP : 0, UXT = OFF_TB;
+
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+        const int t0 = t_begin + c * kC;
+        const int len = min(kC, t_end - t0);
+        const int cur = c & 1, prev = cur ^ 1;
+        const int ch = tid & 127, rh = tid >> 7;
+
+        // ===== E: cumulative log decay, reference point, gated operands =====
+        bool ok = mbar_wait(&bars[0], ph_qkg, 1);
+        ph_qkg ^= 1;
+        if (tid == 0) pend_qkg = false;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        const float* sG = reinterpret_cast<const float*>(sm + OFF_G);
+        float bl[32];
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = rh * 32 + j;
+                const float gv = (r < len) ? fmaxf(sG[r * kD + ch], kGateFloor) : 0.f;
+                acc += gv;
+                bl[j] = acc;
+            }
+            sCarry[rh * 128 + ch] = acc;
+        }
+        if (tid < 64) sBeta[tid] = (tid < len) ? p.beta[size_t(t0 + tid) * H + h] : 0.f;
+        const float b0 = (len > 0) ? fmaxf(sG[ch], kGateFloor) : 0.f;
+        __syncthreads();
+        const float bC = sCarry[ch] + sCarry[128 + ch];
+        const float carry = rh ? sCarry[ch] : 0.f;
+        const bool fast = __syncthreads_and((b0 - bC) <= kRangeMax) != 0;
+        const float m = 0.5f * (b0 + bC);
+        const float mp = fast ? m : 0.f, mk = fast ? m : bC;
+        if (!fast) {  // keep b for the exact A / P (g is dead once bl holds it)
+            float* sB = reinterpret_cast<float*>(sm + OFF_G);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sB[(rh * 32 + j) * kD + ch] = bl[j] + carry;
+        }
+        {
+            const uint8_t* sQb = sm + OFF_Q;
+            const uint8_t* sKb = sm + OFF_K;
+            const uint32_t box = uint32_t(ch >> 6) * 8192u;
+#pragma unroll
+            for (int jj = 0; jj < 32; jj += 8) {
+                uint32_t pk[4], pq[4], pm[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float kv[2], qv[2], e1[2], e2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int j = jj + e + u, r = rh * 32 + j;
+                        const bool valid = r < len;
+                        const float b = bl[j] + carry;
+                        const uint32_t off = box + sw128_off(r, ch & 63);
+                        kv[u] = valid ? bf16_at(sKb, off) : 0.f;
+                        qv[u] = (!kSummary && valid) ? bf16_at(sQb, off) * p.scale : 0.f;
+                        e1[u] = __expf(b - mp);
+                        e2[u] = __expf(mk - b);
+                    }
+                    pk[e >> 1] = pack_bf16x2(kv[0] * e1[0], kv[1] * e1[1]);
+                    pq[e >> 1] = pack_bf16x2(qv[0] * e1[0], qv[1] * e1[1]);
+                    pm[e >> 1] = pack_bf16x2(kv[0] * e2[0], kv[1] * e2[1]);
+                }
+                const int j8 = (rh * 32 + jj) >> 3;
+                st_shared_v4(sbase + OFF_KP + sw128_chunk(ch, j8), pk[0], pk[1], pk[2], pk[3]);
+                if (!kSummary) st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), pq[0], pq[1], pq[2], pq[3]);
+                st_shared_v4(sbase + OFF_KM + sw128_chunk(ch, j8), pm[0], pm[1], pm[2], pm[3]);
+            }
+        }
+        if (tid < 128) {
+            sPreOp[ch] = __expf(mp);
+            sPreAcc[ch] = __expf(mk);
+            sPost[cur * 128 + ch] = __expf(bC - mk);
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // ===== A (scaled by beta, strictly lower) and P (lower incl. diagonal) =====
+        if (fast) {
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : 16384u, 1024);
+                    const uint64_t b = sdesc_sw128(sbase + OFF_KM + ks * 2048, 8192, 1024);
+                    umma_bf16(tbase + TM_AP, a, b, id_ap, ks > 0);
+                }
+                umma_commit(&bars[2]);
+            }
+            ok = mbar_wait(&bars[2], ph_mma, 2);
+            ph_mma ^= 1;
+            tc_fence_after();
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            float vals[32];
+            tmem_ld16(tbase + TM_AP + lane_off + half * 32, vals);
+            tmem_ld16(tbase + TM_AP + lane_off + half * 32 + 16, vals + 16);
+            tmem_wait_ld();
+            if (vrow < 64) {
+                const float br = sBeta[vrow];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int i = half * 32 + j;
+                    sA[vrow * 64 + i] = (i < vrow) ? br * vals[j] : 0.f;
+                }
+            } else if (!kSummary) {
+                const int r = vrow - 64;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i0 = half * 32 + q4 * 8 + 2 * u;
+                        w[u] = pack_bf16x2(i0 <= r ? vals[q4 * 8 + 2 * u] : 0.f,
+                                           i0 + 1 <= r ? vals[q4 * 8 + 2 * u + 1] : 0.f);
+                    }
+                    st_shared_v4(sbase + OFF_P + sw128_chunk(r, half * 4 + q4), w[0], w[1], w[2], w[3]);
+                }
+            }
+        } else {
+            // Exact fallback: one exp per (r, i, c) term, all exponents <= 0.
+            const float* sB = reinterpret_cast<const float*>(sm + OFF_G);
+            const uint8_t* sQb = sm + OFF_Q;
+            const uint8_t* sKb = sm + OFF_K;
+            for (int e = tid; e < 64 * 64; e += 256) sA[e] = 0.f;
+            if (!kSummary)
+                for (int e = tid; e < 512; e += 256) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
+            __syncthreads();
+            for (int pidx = tid; pidx < 64 * 65 / 2; pidx += 256) {
+                int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
+                while (r * (r + 1) / 2 > pidx) --r;
+                while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
+                const int i = pidx - r * (r + 1) / 2;
+                float sa = 0.f, sp = 0.f;
+                if (r < len) {
+                    for (int cc = 0; cc < kD; ++cc) {
+                        const float f = __expf(sB[r * kD + cc] - sB[i * kD + cc]);
+                        const uint32_t offr = uint32_t(cc >> 6) * 8192u + sw128_off(r, cc & 63);
+                        const uint32_t offi = uint32_t(cc >> 6) * 8192u + sw128_off(i, cc & 63);
+                        const float ki = bf16_at(sKb, offi) * f;
+                        sa += bf16_at(sKb, offr) * ki;
+                        if (!kSummary) sp += bf16_at(sQb, offr) * ki;
+                    }
+                }
+                if (i < r) sA[r * 64 + i] = sBeta[r] * sa;
+                if (!kSummary)
+                    *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) =
+                        __float2bfloat16_rn(sp * p.scale);
+            }
+        }
+        __syncthreads();
+
+        // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
+        if (tid < 64) {  // 16x16 diagonal blocks: thread (block I, column jc)
+            const int I = tid >> 4, jc = tid & 15, base = 16 * I;
+            float tcol[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float s = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < r; ++s2) s -= sA[(base + r) * 64 + base + s2] * tcol[s2];
+                tcol[r] = (r >= jc) ? s : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sT[(base + r) * 64 + base + jc] = tcol[r];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int d = 1; d <= 3; ++d) {  // blocks (I, J) with I - J = d:  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+            const int nb = 4 - d;
+            for (int e = tid; e < nb * 256; e += 256) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, i = e & 15;
+                float s = 0.f;
+                for (int kk = 16 * J; kk < 16 * I; ++kk) s += sA[(16 * I + r) * 64 + kk] * sT[kk * 64 + 16 * J + i];
+                sX[e] = s;
+            }
+            __syncthreads();
+            for (int e = tid; e < nb * 256; e += 256) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, i = e & 15;
+                float s = 0.f;
+                for (int j2 = 0; j2 <= r; ++j2) s += sT[(16 * I + r) * 64 + 16 * I + j2] * sX[(J << 8) + j2 * 16 + i];
+                sT[(16 * I + r) * 64 + 16 * J + i] = -s;
+            }
+            __syncthreads();
+        }
+        for (int e = tid; e < 64 * 8; e += 256) {  // (T diag(beta)) as bf16 rows [r][i]
+            const int r = e >> 3, j = e & 7;
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i0 = 8 * j + 2 * u;
+                w[u] = pack_bf16x2(i0 <= r ? sT[r * 64 + i0] * sBeta[i0] : 0.f,
+                                   i0 + 1 <= r ? sT[r * 64 + i0 + 1] * sBeta[i0 + 1] : 0.f);
+            }
+            st_shared_v4(sbase + OFF_TB + sw128_chunk(r, j), w[0], w[1], w[2], w[3]);
+        }
+        fence_async_smem();
+        ok = mbar_wait(&bars[1], ph_v, 3);
+        ph_v ^= 1;
+        if (tid == 0) pend_v = false;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+
+        // ===== W^T = Kp^T (T beta)^T and U^T = V^T (T beta)^T =====
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t bt = sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024);
+                umma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_KP + ks * 32, 16, 1024), bt, id_w, ks > 0);
+                umma_bf16(tbase + TM_U, sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), bt, id_u, ks > 0);
+            }
+            umma_commit(&bars[2]);
+            if (c + 1 < nchunks) {  // q, k, g of this chunk are consumed
+                issue_qkg(c + 1);
+                pend_qkg = true;
+            }
+        }
+
+        // ===== S frame: S <- S * post(prev) ; operand = S * preop ; TMEM = S * preacc =====
+        {
+            auto frame = [&](uint32_t tcol, uint32_t st_off0, uint32_t st_off1) {
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    const int k0 = half * 64 + cb * 16;
+                    float x[16];
+                    tmem_ld16(tbase + tcol + lane_off + k0, x);
+                    tmem_wait_ld();
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        const float x0 = x[j] * sPost[prev * 128 + k0 + j];
+                        const float x1 = x[j + 1] * sPost[prev * 128 + k0 + j + 1];
+                        pk[j >> 1] = pack_bf16x2(x0 * sPreOp[k0 + j], x1 * sPreOp[k0 + j + 1]);
+                        x[j] = x0 * sPreAcc[k0 + j];
+                        x[j + 1] = x1 * sPreAcc[k0 + j + 1];
+                    }
+                    tmem_st16(tbase + tcol + lane_off + k0, x);
+                    const uint32_t dst = sbase + (half ? st_off1 : st_off0);
+                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2), pk[0], pk[1], pk[2], pk[3]);
+                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2 + 1), pk[4], pk[5], pk[6], pk[7]);
+                }
+            };
+            frame(TM_S, OFF_ST, OFF_ST + 16384);
+            if (kSummary) frame(TM_X, XT0, XT1);
+            tmem_wait_st();
+        }
+        ok = mbar_wait(&bars[2], ph_mma, 4);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        if (tid == 0 && c + 1 < nchunks) {  // V of this chunk is consumed
+            issue_v(c + 1);
+            pend_v = true;
+        }
+        {  // -W^T -> smem (lane = key channel k, 32 tokens per thread)
+            float w[32];
+            tmem_ld16(tbase + TM_W + lane_off + half * 32, w);
+            tmem_ld16(tbase + TM_W + lane_off + half * 32 + 16, w + 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                st_shared_v4(sbase + OFF_WN + sw128_chunk(vrow, half * 4 + q4),
+                             pack_bf16x2(-w[q4 * 8 + 0], -w[q4 * 8 + 1]), pack_bf16x2(-w[q4 * 8 + 2], -w[q4 * 8 + 3]),
+                             pack_bf16x2(-w[q4 * 8 + 4], -w[q4 * 8 + 5]), pack_bf16x2(-w[q4 * 8 + 6], -w[q4 * 8 + 7]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ===== U~^T = U^T - S'^T W^T ;  O^T = S'^T Qp  (or U_X~^T = -X'^T W^T) =====
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = sdesc_sw128(sbase + OFF_ST + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                umma_bf16(tbase + TM_U, a, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, 1);
+                if (!kSummary) {
+                    umma_bf16(tbase + TM_O, a, sdesc_sw128(sbase + OFF_QP + ks * 2048, 8192, 1024), id_so, ks > 0);
+                } else {
+                    const uint64_t ax = sdesc_sw128(sbase + ((ks >> 2) ? XT1 : XT0) + (ks & 3) * 32, 16, 1024);
+                    umma_bf16(tbase + TM_O, ax, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, ks > 0);
+                }
+            }
+            umma_commit(&bars[2]);
+        }
+        ok = mbar_wait(&bars[2], ph_mma, 5);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        {  // U~^T (and U_X~^T) -> smem, lane = value channel, 32 tokens per thread
+            auto spill = [&](uint32_t tcol, uint32_t dst_off) {
+                float u[32];
+                tmem_ld16(tbase + tcol + lane_off + half * 32, u);
+                tmem_ld16(tbase + tcol + lane_off + half * 32 + 16, u + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    st_shared_v4(sbase + dst_off + sw128_chunk(vrow, half * 4 + q4),
+                                 pack_bf16x2(u[q4 * 8 + 0], u[q4 * 8 + 1]), pack_bf16x2(u[q4 * 8 + 2], u[q4 * 8 + 3]),
+                                 pack_bf16x2(u[q4 * 8 + 4], u[q4 * 8 + 5]), pack_bf16x2(u[q4 * 8 + 6], u[q4 * 8 + 7]));
+            };
+            spill(TM_U, OFF_UT);
+            if (kSummary) spill(TM_O, UXT);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ===== O^T += U~^T P^T ;  S^T += U~^T Km  (X^T += U_X~^T Km) =====
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t a = sdesc_sw128(sbase + OFF_UT + ks * 32, 16, 1024);
+                if (!kSummary)
+                    umma_bf16(tbase + TM_O, a, sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024), id_po, 1);
+                umma_bf16(tbase + TM_S, a, sdesc_sw128(sbase + OFF_KM + ks * 32, 16, 1024), id_s, 1);
+                if (kSummary)
+                    umma_bf16(tbase + TM_X, sdesc_sw128(sbase + UXT + ks * 32, 16, 1024),
+                              sdesc_sw128(sbase + OFF_KM + ks * 32, 16, 1024), id_s, 1);
+            }
+            umma_commit(&bars[2]);
+        }
+        ok = mbar_wait(&bars[2], ph_mma, 6);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+
+        if (!kSummary) {  // O^T -> o[t0 + r, h, v]
+            float ov[32];
+            tmem_ld16(tbase + TM_O + lane_off + half * 32, ov);
+            tmem_ld16(tbase + TM_O + lane_off + half * 32 + 16, ov + 16);
+            tmem_wait_ld();
+            OutT* o = static_cast<OutT*>(p.o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = half * 32 + j;
+                if (r < len) o[(size_t(t0 + r) * H + h) * kD + vrow] = from_f32<OutT>(ov[j]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (!aborted) {
+        // ---- end state: S = S^T(TMEM) * post(last chunk)
+        const int last = (nchunks - 1) & 1;
+        float* dstS = nullptr;
+        float* dstX = nullptr;
+        if (kSummary) {
+            dstS = p.segN + (size_t(item_id) * H + h) * (kD * kD);
+            dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
+        } else if (it.g == it.G - 1 && p.final_state) {
+            dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
+        }
+        tc_fence_after();
+        auto store = [&](uint32_t tcol, float* dst) {
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                const int k0 = half * 64 + cb * 16;
+                float x[16];
+                tmem_ld16(tbase + tcol + lane_off + k0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) dst[size_t(k0 + j) * kD + vrow] = x[j] * sPost[last * 128 + k0 + j];
+            }
+        };
+        if (dstS) store(TM_S, dstS);
+        if (dstX) store(TM_X, dstX);
+    } else if (tid == 0) {
+        // let copies still in flight land before the shared memory is released
+        if (pend_qkg) mbar_wait(&bars[0], ph_qkg, 7);
+        if (pend_v) mbar_wait(&bars[1], ph_v, 7);
+        mbar_wait(&bars[2], ph_mma, 7);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// ---------------------------------------------------------------- plan
+// One CTA: per sequence n, G_n = max(1, ceil(chunks_n / L)) segments; writes the
+// segment table in sequence order and the item count.
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, int T, int L, SegItem* items,
+                                                    int* n_items, int max_items) {
+    using Scan = cub::BlockScan<int, 1024>;
+    __shared__ typename Scan::TempStorage tmp;
+    __shared__ int s_base;
+    if (threadIdx.x == 0) s_base = 0;
+    __syncthreads();
+    for (int n0 = 0; n0 < N; n0 += 1024) {
+        const int n = n0 + threadIdx.x;
+        int sb = 0, se = 0, G = 0;
+        if (n < N) {
+            sb = cu ? cu[n] : n * T;
+            se = cu ? cu[n + 1] : (n + 1) * T;
+            const int nch = (se - sb + kC - 1) / kC;
+            G = nch > 0 ? (nch + L - 1) / L : 1;
+        }
+        int off = 0, tot = 0;
+        Scan(tmp).ExclusiveSum(G, off, tot);
+        off += s_base;
+        if (n < N) {
+            for (int g = 0; g < G; ++g) {
+                const int id = off + g;
+                if (id >= max_items) break;
+                SegItem s;
+                s.seq = n;
+                s.tok_begin = int(min((long long)se, sb + (long long)g * L * kC));
+                s.tok_end = int(min((long long)se, sb + (long long)(g + 1) * L * kC));
+                s.g = g;
+                s.G = G;
+                s.first = off;
+                s.pad0 = s.pad1 = 0;
+                items[id] = s;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) s_base += tot;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *n_items = min(s_base, max_items);
+}
+
+// ---------------------------------------------------------------- combine
+// Chains the segment maps of one (sequence, head, 8-column slice):
+// S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1.
+__global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const float* init,
+                                                      const float* segN, const float* segX, float* segS, int H) {
+    const int item = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
+    if (item >= *n_items) return;
+    const SegItem it = items[item];
+    if (it.g != 0 || it.G < 2) return;
+    __shared__ float sS[kD][8];
+    const int tid = threadIdx.x;
+    const int k = tid >> 1, j0 = (tid & 1) * 4;
+    for (int e = tid; e < kD * 8; e += 256) {
+        const int kk = e >> 3, jj = e & 7;
+        const float s0 = init ? init[(size_t(it.seq) * H + h) * (kD * kD) + size_t(kk) * kD + 8 * z + jj] : 0.f;
+        sS[kk][jj] = s0;
+        segS[(size_t(item) * H + h) * (kD * kD) + size_t(kk) * kD + 8 * z + jj] = s0;
+    }
+    __syncthreads();
+    for (int g = 0; g + 1 < it.G; ++g) {
+        const size_t base = (size_t(item + g) * H + h) * (kD * kD);
+        const float4* Xr = reinterpret_cast<const float4*>(segX + base + size_t(k) * kD);
+        float acc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] = segN[base + size_t(k) * kD + 8 * z + j0 + u];
+#pragma unroll 4
+        for (int k4 = 0; k4 < kD / 4; ++k4) {
+            const float4 x = Xr[k4];
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] += xs[w] * sS[4 * k4 + w][j0 + u];
+            }
+        }
+        __syncthreads();
+        const size_t out = (size_t(item + g + 1) * H + h) * (kD * kD) + size_t(k) * kD + 8 * z + j0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            sS[k][j0 + u] = acc[u];
+            segS[out + u] = acc[u];
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- prep
+// One warp per (token, head) row: optional L2 normalisation of q / k and a
+// cast to bf16 (used for fp32 inputs or l2norm_qk).
+template <typename T>
+__global__ void prep_rows_kernel(const T* __restrict__ src, __nv_bfloat16* __restrict__ dst, long long rows,
+                                 int normalize) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float x[4];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        x[u] = to_f32(src[row * kD + lane * 4 + u]);
+        ss += x[u] * x[u];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float f = normalize ? rsqrtf(ss + 1e-6f) : 1.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) dst[row * kD + lane * 4 + u] = __float2bfloat16_rn(x[u] * f);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [Ttot, H, 128] token tensor as a 3-D map (c, h, t); box = (bc, 1, 64).
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int H, long long Ttot,
+                     int bc, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(H), cuuint64_t(Ttot)};
+    cuuint64_t strides[2] = {cuuint64_t(kD) * esize, cuuint64_t(H) * kD * esize};
+    cuuint32_t box[3] = {cuuint32_t(bc), 1, cuuint32_t(kC)};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+struct ChunkPlan {
+    int N, L, max_items;
+    long long Ttot;
+    bool scan;
+    size_t off_items, off_count, off_segN, off_segX, off_segS, off_q, off_k, off_v, total;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2norm, bool varlen, int nsm) {
+    ChunkPlan pl{};
+    pl.N = varlen ? num_seqs : B;
+    pl.Ttot = varlen ? (long long)T : (long long)B * T;
+    const long long chunks_bound = (pl.Ttot + kC - 1) / kC + pl.N;
+    const long long pairs = (long long)pl.N * H;
+    int L = 1 << 30;
+    if (pairs > 0 && pairs * 3 <= nsm) {
+        const long long G = nsm / pairs;  // segments per sequence
+        const long long per_seq = (chunks_bound + pl.N - 1) / pl.N;
+        L = int((per_seq + G - 1) / G);
+        if (L < 1) L = 1;
+        if (per_seq < 3 * (long long)L) L = 1 << 30;  // too short to pay for the summary pass
+    }
+    pl.L = L;
+    pl.scan = L < (1 << 30);
+    pl.max_items = int(pl.N + (pl.scan ? (chunks_bound + L - 1) / L : 0));
+    size_t off = 0;
+    pl.off_items = off; off = up256(off + sizeof(SegItem) * size_t(pl.max_items));
+    pl.off_count = off; off = up256(off + 16);
+    const size_t st = size_t(pl.max_items) * H * kD * kD * sizeof(float);
+    pl.off_segN = off; off = up256(off + (pl.scan ? st : 0));
+    pl.off_segX = off; off = up256(off + (pl.scan ? st : 0));
+    pl.off_segS = off; off = up256(off + (pl.scan ? st : 0));
+    const size_t tok = size_t(pl.Ttot) * H * kD * sizeof(__nv_bfloat16);
+    const bool need_qk = (dtype == KDA_FP32) || l2norm;
+    pl.off_q = off; off = up256(off + (need_qk ? tok : 0));
+    pl.off_k = off; off = up256(off + (need_qk ? tok : 0));
+    pl.off_v = off; off = up256(off + (dtype == KDA_FP32 ? tok : 0));
+    pl.total = off;
+    return pl;
+}
+
+template <bool S, typename O>
+static cudaError_t set_smem_attr() {
+    static bool done = false;
+    if (done) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(chunk_kernel<S, O>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
+int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
+                     int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
+                     const char** why) {
+    const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
+    if (ws_bytes < pl.total || (pl.total > 0 && ws == nullptr)) {
+        *why = "workspace smaller than kda_chunk_fwd_workspace()";
+        return KDA_ERR_WORKSPACE;
+    }
+    if (pl.N == 0 || H == 0) return KDA_OK;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    SegItem* items = reinterpret_cast<SegItem*>(w + pl.off_items);
+    int* n_items = reinterpret_cast<int*>(w + pl.off_count);
+    const long long rows = pl.Ttot * H;
+
+    const void *qb = q, *kb = k, *vb = v;
+    if (dtype == KDA_FP32 || l2norm) {
+        const unsigned grid = unsigned((rows + 7) / 8);
+        __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(w + pl.off_q);
+        __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(w + pl.off_k);
+        if (rows > 0) {
+            if (dtype == KDA_FP32) {
+                prep_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(q), dq, rows, l2norm);
+                prep_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(k), dk, rows, l2norm);
+            } else {
+                prep_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), dq,
+                                                                          rows, l2norm);
+                prep_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), dk,
+                                                                          rows, l2norm);
+            }
+        }
+        qb = dq;
+        kb = dk;
+        if (dtype == KDA_FP32) {
+            __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(w + pl.off_v);
+            if (rows > 0)
+                prep_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(v), dv, rows, 0);
+            vb = dv;
+        }
+    }
+
+    CUtensorMap mq, mk, mv, mg;
+    const long long Tmap = pl.Ttot > 0 ? pl.Ttot : 1;
+    if (!make_map(&mq, qb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, Tmap, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        *why = "cuTensorMapEncodeTiled failed";
+        return KDA_ERR_CUDA;
+    }
+
+    cudaEvent_t* ev = g_trace_events;
+    if (ev) cudaEventRecord(ev[0], stream);
+    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items);
+    if (ev) cudaEventRecord(ev[1], stream);
+
+    ChunkArgs a{};
+    a.beta = beta;
+    a.init_state = init;
+    a.final_state = fin;
+    a.o = o;
+    a.items = items;
+    a.n_items = n_items;
+    a.segN = reinterpret_cast<float*>(w + pl.off_segN);
+    a.segX = reinterpret_cast<float*>(w + pl.off_segX);
+    a.segS = reinterpret_cast<const float*>(w + pl.off_segS);
+    a.H = H;
+    a.scale = scale;
+    const dim3 grid(unsigned(pl.max_items), unsigned(H));
+    if (pl.scan) {
+        if (set_smem_attr<true, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
+        chunk_kernel<true, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+        if (ev) cudaEventRecord(ev[2], stream);
+        combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), 16), 256, 0, stream>>>(
+            items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
+        if (ev) cudaEventRecord(ev[3], stream);
+    } else if (ev) {
+        cudaEventRecord(ev[2], stream);
+        cudaEventRecord(ev[3], stream);
+    }
+    if (dtype == KDA_FP32) {
+        if (set_smem_attr<false, float>() != cudaSuccess) return KDA_ERR_CUDA;
+        chunk_kernel<false, float><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+    } else {
+        if (set_smem_attr<false, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
+        chunk_kernel<false, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+    }
+    if (ev) cudaEventRecord(ev[4], stream);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *why = cudaGetErrorString(e);
+        return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
+    return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total;
+}
+
+}  // namespace kda

@@ -1,0 +1,199 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library.
+ *
+ * The operation (Kimi Delta Attention, "KDA"), per head with a d_k x d_v state S
+ * (d_k = d_v = 128 here), for tokens t = 1..T of one sequence:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T (scale * q_t)
+ *
+ * with a per-channel decay alpha_t = exp(g_t) in [0,1]^{d_k} and a scalar write
+ * strength beta_t.  Source: "Kimi Linear: An Expressive, Efficient Attention
+ * Architecture" (research notes on arXiv 2510.26692), section Method, "From
+ * Linear Attention to KDA", eq. KDA and its residual reading
+ * S~ = Diag(alpha_t) S_{t-1}, S_t = S~ + beta_t k_t (v_t - S~^T k_t)^T.
+ * The state's rows are key channels (Diag(alpha) scales rows); scale = 1 is the
+ * pages' o_t = S_t^T q_t.
+ *
+ * Conventions for every entry point below:
+ *  - All tensor pointers are DEVICE pointers owned by the caller (allocated by
+ *    whatever allocator it uses); the library never allocates, frees or keeps
+ *    them.  Scratch memory comes only from the caller's `workspace`.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Arguments are validated on the host before any launch;
+ *    a rejected call launches nothing and returns a status code.  No entry
+ *    point throws, aborts or prints.
+ *  - Token tensors are row-major with the head dim fastest: [B, T, H, 128]
+ *    (dense) or [1, Ttot, H, 128] (packed, with cu_seqlens).  States are fp32
+ *    [N, H, 128 (key channel), 128 (value channel)], value channel fastest.
+ *  - Pointers must be 16-byte aligned.  Outputs must not alias inputs except
+ *    where stated (the decode state is updated in place).
+ *  - Device-side waits are bounded: a kernel that waits too long gives up,
+ *    records KDA_ERR_TIMEOUT in a device status word and exits cleanly; read it
+ *    with kda_device_status() (which synchronises `stream`).
+ *  - The caller's current CUDA device must be the device that holds the
+ *    pointers.
+ */
+#ifndef KDA_B200_H_
+#define KDA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* NULL where not allowed, bad size, misaligned pointer */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. head dim != 128) */
+    KDA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than the matching *_workspace() query */
+    KDA_ERR_CUDA = 4,         /* a CUDA runtime / driver call or kernel launch failed */
+    KDA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see kda_device_status) */
+} kda_status;
+
+typedef enum {
+    KDA_BF16 = 0,
+    KDA_FP32 = 1
+} kda_dtype;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *kda_status_string(int status);
+
+/* Head dimension this build supports (d_k = d_v): 128. */
+int kda_head_dim(void);
+
+/* Detail of the last host-side rejection or CUDA error on this thread
+ * (static thread-local storage; empty string when none). */
+const char *kda_last_error(void);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device: KDA_OK, or KDA_ERR_TIMEOUT if any kernel of this library gave
+ * up a bounded wait since the last call, or KDA_ERR_CUDA if the sync failed. */
+int kda_device_status(void *stream);
+
+/* Optional tracing hook for kda_chunk_fwd.  When `events` is non-NULL it must
+ * point to 5 cudaEvent_t created by the caller on the current device; every
+ * later kda_chunk_fwd call on this thread records them on its stream around
+ * its kernels: [0] before the plan kernel, [1] after it, [2] after the segment
+ * summary pass (same as [1] when the sequence is not segmented), [3] after the
+ * combine pass, [4] after the output pass.  Pass NULL to stop.  The events stay
+ * owned by the caller. */
+int kda_set_trace_events(void *events, int n_events);
+
+/* ------------------------------------------------------------------------
+ * kda_chunk_fwd -- chunkwise-parallel prefill.
+ *
+ * Computes o and the final state of the recurrence above over whole sequences
+ * (chunks of 64 tokens; "Kimi Linear: An Expressive, Efficient Attention
+ * Architecture", section "Chunkwise Algorithm": per-channel decay and rank-1
+ * corrections unrolled inside a chunk, WY representation, UT transform, only
+ * the fixed-size state crossing chunks; the inverse (I + A)^{-1} by forward
+ * substitution, "Kimi Linear" news rewrite, section on the hardware-efficient
+ * chunkwise algorithm).  The result is the recurrence's, up to rounding.
+ *
+ *   q, k      [B,T,H,128] (dense) or [1,Ttot,H,128] (packed); dtype bf16 or fp32.
+ *             With l2norm_qk != 0 each (token, head) row of q and k is first
+ *             normalised to unit L2 norm (x / sqrt(sum x^2 + 1e-6)).
+ *   v         same shape and dtype as q.
+ *   g         fp32, same shape: log of the per-channel decay (alpha = exp(g)),
+ *             expected <= 0.  Values below -1e4 are treated as -1e4 (alpha = 0
+ *             in fp32).
+ *   beta      fp32 [B,T,H] (or [1,Ttot,H]).
+ *   initial_state  fp32 [N,H,128,128] or NULL (zero state).
+ *   final_state    fp32 [N,H,128,128] or NULL (not written).  May alias
+ *                  initial_state.
+ *   o         output, same shape and dtype as q.
+ *   cu_seqlens     NULL for dense input (N = B sequences of T tokens; then
+ *                  num_seqs must be 0), or a device int32 [num_seqs+1] of
+ *                  non-decreasing token offsets with cu_seqlens[0] = 0 and
+ *                  cu_seqlens[num_seqs] = T (T = total packed tokens); then B
+ *                  must be 1 and N = num_seqs >= 1.  Empty sequences are allowed.
+ *                  The offsets are read on the device only (never copied back).
+ *   scale     multiplies q (1.0 = o_t = S_t^T q_t).
+ *   workspace      device scratch of at least kda_chunk_fwd_workspace(...)
+ *                  bytes, 256-byte aligned; contents need not be initialised
+ *                  and are clobbered.
+ *
+ * Tensor cores compute the chunk contractions with bf16 operands and fp32
+ * accumulation; the state is carried in fp32.  fp32 inputs are rounded to
+ * bf16 where they feed the tensor cores.
+ */
+/* Workspace bytes for a kda_chunk_fwd call with the same B, T, H, num_seqs
+ * (0 = dense), dtype and l2norm_qk, on the current device. */
+size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk);
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *initial_state, float *final_state, void *o, const int32_t *cu_seqlens,
+                  int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * kda_decode_step -- one recurrent step for B sequences (one token each).
+ *
+ * Residual form, "Kimi Linear: An Expressive, Efficient Attention
+ * Architecture", section Method (S~ = Diag(alpha) S; S = S~ + beta k (v - S~^T
+ * k)^T) and section "Code Verification" (the naive recurrence multiplies by
+ * exp(g), then writes the residual); decode uses this recurrent form (section
+ * "Training and Inference").  Each head's state is read once and written once.
+ *
+ *   q, k, v   [B,H,128], dtype bf16 or fp32 (l2norm_qk as for kda_chunk_fwd).
+ *   g         fp32 [B,H,128] log decay;  beta fp32 [B,H].
+ *   state     fp32 [B,H,128,128], updated IN PLACE.
+ *   o         [B,H,128], same dtype as q; o = S_new^T (scale * q).
+ * All arithmetic is fp32 on CUDA cores.  No workspace.
+ */
+int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    float *state, void *o, int B, int H, int dtype, float scale, int l2norm_qk,
+                    void *stream);
+
+/* ------------------------------------------------------------------------
+ * kda_layer_fwd -- the KDA layer around the operator (forward).
+ *
+ * "Kimi Linear: An Expressive, Efficient Attention Architecture", section
+ * "Neural Parameterization" and "Code Verification": bias-free Q/K/V
+ * projections; depthwise causal ShortConv (kernel 4) then SiLU on q, k, v;
+ * L2 norm of q and k; per-channel decay alpha = exp(-softplus(W_aup W_adown x))
+ * (rank-128 low-rank projection); beta = sigmoid(W_b x); KDA (scale 1); per-head
+ * RMSNorm (eps 1e-5, weight norm_w) times sigmoid(W_gup W_gdown x); output
+ * projection.  Packed sequences: the convolution restarts from zero history at
+ * every cu_seqlens start.
+ *
+ * All weights are bf16 row-major "out x in" (y = x W^T) except conv_* and
+ * norm_w:
+ *   W_in    [3*H*128 + 2*rank + H, d_model]: rows are, in order, W_q, W_k, W_v
+ *           (H*128 each), W_adown (rank), W_gdown (rank), W_b (H).
+ *   W_aup   [H*128, rank];  W_gup [H*128, rank];
+ *   conv_w  bf16 [3*H*128, 4]: depthwise taps for the q, k, v channels; tap j
+ *           multiplies x[t-3+j];
+ *   norm_w  fp32 [128];     W_o [d_model, H*128].
+ *   x       bf16 [total_tokens, d_model];  y bf16 [total_tokens, d_model].
+ *   cu_seqlens  device int32 [num_seqs+1] (required);
+ *   initial_state / final_state as in kda_chunk_fwd (N = num_seqs).
+ * Projections run on cuBLASLt (plain bf16 GEMMs, fp32 accumulate); everything
+ * else runs in this library's kernels.
+ */
+typedef struct {
+    const void *W_in;
+    const void *W_aup;
+    const void *W_gup;
+    const void *conv_w;
+    const float *norm_w;
+    const void *W_o;
+    int d_model;
+    int H;
+    int rank;
+} kda_layer_weights;
+
+size_t kda_layer_fwd_workspace(int total_tokens, int d_model, int H, int rank, int num_seqs);
+
+int kda_layer_fwd(const void *x, const kda_layer_weights *w, const int32_t *cu_seqlens, int num_seqs,
+                  int total_tokens, const float *initial_state, float *final_state, void *y,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H_ */

@@ -1,0 +1,134 @@
+"""kda_chunk_fwd vs the fp64 oracle recurrence.
+
+Tolerance (from the operator's precision: bf16 tensor-core operands, fp32
+accumulation and fp32 state): relative L2 error <= 1e-2 on o and on the final
+state, over the whole tensor.  The oracle's fp64 o is compared directly (the
+GPU rounds o to bf16 once, ~2e-3 relative)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+def run_both(kda, inp, scale=1.0, l2=False, heads=None):
+    q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
+    cu = inp.get("cu_seqlens")
+    s0 = inp.get("s0")
+    o, fs = kda.chunk_fwd(q.cuda(), k.cuda(), v.cuda(), g.cuda(), beta.cuda(),
+                          initial_state=None if s0 is None else s0.cuda(),
+                          cu_seqlens=None if cu is None else cu.cuda(), scale=scale, l2norm_qk=l2)
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    if heads is not None:  # compare a subset of heads (sliced before leaving the device)
+        hs = torch.as_tensor(heads) if isinstance(heads, list) else torch.arange(q.shape[2])[heads]
+        hs = hs.to(q.device)
+        q, k, v, g, beta = (t.index_select(2, hs) for t in (q, k, v, g, beta))
+        o = o.index_select(2, hs.to(o.device))
+        fs = fs.index_select(1, hs.to(fs.device))
+        s0 = None if s0 is None else s0.index_select(1, hs.to(s0.device))
+    qn, kn = f64(q), f64(k)
+    if l2:
+        qn = qn / np.sqrt((qn * qn).sum(-1, keepdims=True) + 1e-6)
+        kn = kn / np.sqrt((kn * kn).sum(-1, keepdims=True) + 1e-6)
+    if cu is None:
+        o_ref, s_ref = oracle.kda_recurrent(qn, kn, f64(v), f64(g), f64(beta), s0=f64(s0), scale=scale)
+        o_got = f64(o)
+    else:
+        o_ref, s_ref = oracle.kda_recurrent(qn[0], kn[0], f64(v)[0], f64(g)[0], f64(beta)[0], s0=f64(s0),
+                                            cu=cu.cpu().numpy(), scale=scale)
+        o_got = f64(o)[0]
+    s_got = f64(fs)
+    assert np.isfinite(o_got).all() and np.isfinite(s_got).all()
+    return rel_l2(o_got, o_ref), rel_l2(s_got, s_ref)
+
+
+def test_oracle_sized_fp32(kda):
+    """B=1, H=2, T=256 fp32, zero initial state (the oracle-sized workload)."""
+    inp = synth.op_inputs(**synth.ORACLE_SIZED)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 1), (1, 1, 2), (2, 63, 2), (1, 65, 3), (2, 200, 3), (3, 130, 5)])
+def test_small_shapes_bf16_with_state(kda, B, T, H):
+    inp = synth.op_inputs(B=B, H=H, T=T, s0_std=0.02, seed=100 + T)
+    eo, es = run_both(kda, inp, scale=0.9)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_no_segment_scan_path(kda):
+    """Enough (sequence, head) pairs that every CTA runs a whole sequence."""
+    inp = synth.op_inputs(B=4, H=40, T=300, s0_std=0.02, seed=7)
+    eo, es = run_both(kda, inp, heads=slice(0, 40, 7))
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_strong_decay_exact_fallback(kda):
+    """Gates ~20x stronger: the in-chunk decay range exceeds the factored
+    path's bound, so chunks take the exact fallback."""
+    inp = synth.op_inputs(B=1, H=2, T=257, gate_scale=3.0, s0_std=0.02, seed=8)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_mixed_decay_strength(kda):
+    inp = synth.op_inputs(B=1, H=2, T=512, gate_scale=1.0, s0_std=0.02, seed=9)
+    inp["g"][:, 200:300] *= 4.0
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_scalar_gate_gdn_case(kda):
+    inp = synth.op_inputs(B=1, H=4, T=333, s0_std=0.02, seed=10, scalar_gate=True)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_l2norm_in_kernel(kda):
+    inp = synth.op_inputs(B=1, H=2, T=150, s0_std=0.02, seed=12)
+    inp["q"] = (inp["q"].float() * 4.0).bfloat16()
+    inp["k"] = (inp["k"].float() * 0.3).bfloat16()
+    eo, es = run_both(kda, inp, l2=True)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_varlen_with_empty_and_short_sequences(kda):
+    cu = [0, 0, 5, 69, 70, 70, 300, 301, 600]
+    inp = synth.op_inputs(B=len(cu) - 1, H=3, T=cu[-1], s0_std=0.02, seed=13, cu_seqlens=cu)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_final_state_only_and_zero_state(kda):
+    inp = synth.op_inputs(B=2, H=2, T=100, s0_std=None, seed=14)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_deterministic_bits(kda):
+    inp = synth.op_inputs(B=1, H=2, T=700, s0_std=0.02, seed=15)
+    a = [kda.chunk_fwd(*(inp[n].cuda() for n in ("q", "k", "v", "g", "beta")), initial_state=inp["s0"].cuda())
+         for _ in range(2)]
+    assert torch.equal(a[0][0], a[1][0]) and torch.equal(a[0][1], a[1][1])
+
+
+def test_prefill_4k_full(kda):
+    """B=1, H=16, T=4096 bf16 with a random initial state: every head."""
+    inp = synth.op_inputs(**synth.PREFILL_4K)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+
+
+@pytest.mark.slow
+def test_prefill_64k_sampled_heads(kda):
+    """B=1, H=16, T=65536 (the length sweep's largest point), in the launch
+    configuration the bench times; the oracle checks heads 0 and 11."""
+    inp = synth.op_inputs(**synth.prefill_sweep(65536), device="cuda")
+    eo, es = run_both(kda, inp, heads=[0, 11])
+    assert eo < TOL and es < TOL, (eo, es)

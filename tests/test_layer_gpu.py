@@ -1,0 +1,63 @@
+"""kda_layer_fwd vs the fp64 oracle layer.
+
+The GPU path rounds every intermediate activation to bf16 (the projection
+outputs, q/k/v after the convolution, the gate and norm inputs, the KDA
+output), each a relative error of about 2^-9; the oracle keeps fp64
+throughout.  Tolerance: relative L2 <= 1e-2 on y and on the final state."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+def run_layer(kda, d_model, H, Ttot, nseq, rank, seed, s0=True, check_seqs=None):
+    x, W, cu = synth.layer_inputs(d_model=d_model, H=H, Ttot=Ttot, nseq=nseq, rank=rank, seed=seed)
+    S0 = 0.02 * torch.randn((nseq, H, 128, 128), generator=torch.Generator().manual_seed(seed)) if s0 else None
+    dev = torch.device("cuda")
+    Wd = {n: t.to(dev) for n, t in W.items()}
+    packed = kda.pack_layer_weights(Wd)
+    cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
+    y, fs = kda.layer_fwd(x.to(dev), packed, cu_d, initial_state=None if S0 is None else S0.to(dev))
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    Wn = {n: f64(t) for n, t in W.items()}
+    seqs = range(nseq) if check_seqs is None else check_seqs
+    errs = []
+    for n in seqs:
+        t0, t1 = cu[n], cu[n + 1]
+        y_ref, s_ref = oracle.kda_layer(f64(x)[t0:t1], Wn, [0, t1 - t0], H,
+                                        s0=None if S0 is None else f64(S0)[n:n + 1])
+        errs.append((rel_l2(f64(y)[t0:t1], y_ref) if t1 > t0 else 0.0, rel_l2(f64(fs)[n], s_ref[0])))
+    return errs
+
+
+def test_layer_small(kda):
+    errs = run_layer(kda, d_model=256, H=2, Ttot=300, nseq=3, rank=32, seed=21)
+    for ey, es in errs:
+        assert ey < TOL and es < TOL, errs
+
+
+def test_layer_many_short_sequences_no_state(kda):
+    errs = run_layer(kda, d_model=128, H=3, Ttot=200, nseq=9, rank=16, seed=22, s0=False)
+    for ey, es in errs:
+        assert ey < TOL and es < TOL, errs
+
+
+@pytest.mark.slow
+def test_layer_full_size_sampled_sequences(kda):
+    """d_model=2048, H=16, 65536 packed tokens in 8 sequences (rank 128): the
+    oracle checks the two shortest sequences end to end."""
+    cfg = synth.LAYER_65K
+    cu = synth.random_cu_seqlens(cfg["Ttot"], cfg["nseq"], cfg["seed"])
+    lens = np.diff(cu)
+    pick = list(np.argsort(lens)[:2])
+    errs = run_layer(kda, d_model=cfg["d_model"], H=cfg["H"], Ttot=cfg["Ttot"], nseq=cfg["nseq"], rank=cfg["rank"],
+                     seed=cfg["seed"], check_seqs=pick)
+    for ey, es in errs:
+        assert ey < TOL and es < TOL, errs
