@@ -14,7 +14,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkda.so")
+# KDA_LIB may point at another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("KDA_LIB") or os.path.join(_HERE, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
 KDA_BF16, KDA_FP32 = 0, 1
@@ -108,6 +109,9 @@ def set_trace_events(events):
         _trace_keep = None
         _check(_lib.kda_set_trace_events(None, 0), "kda_set_trace_events")
         return
+    for e in events:  # torch creates the CUDA event lazily, on its first record
+        if e.cuda_event == 0:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _trace_keep = (arr, events)
     _check(_lib.kda_set_trace_events(arr, len(events)), "kda_set_trace_events")

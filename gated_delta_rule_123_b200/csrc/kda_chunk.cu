@@ -57,6 +57,24 @@ struct SegItem {
     int pad0, pad1;
 };
 
+// Optional per-stage cycle counters (thread 0 of every CTA), compiled in only
+// with -DKDA_STAGE_TIMING for profiling builds.
+#ifdef KDA_STAGE_TIMING
+__device__ unsigned long long g_stage_cycles[32];
+#define KDA_STAGE(i)                                                                                   \
+    do {                                                                                               \
+        if (tid == 0) {                                                                                \
+            const long long t_ = clock64();                                                            \
+            atomicAdd(&g_stage_cycles[(kSummary ? 16 : 0) + (i)], (unsigned long long)(t_ - ts_));     \
+            ts_ = t_;                                                                                  \
+        }                                                                                              \
+    } while (0)
+#else
+#define KDA_STAGE(i) \
+    do {             \
+    } while (0)
+#endif
+
 constexpr float kRangeMax = 64.f;   // max in-chunk decay range (nats) for the factored path
 constexpr float kGateFloor = -1e4f; // log-gates below this are treated as this
 
@@ -76,7 +94,7 @@ constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S^T (operand copy)
 constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T (also fp32 T scratch)
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_BYTES = 7 * 1024;
-constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES;
 // Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
 
 // TMEM columns (512 allocated): S^T | [A;P] | W^T | U^T | O^T (or U_X^T) | X^T
@@ -96,9 +114,41 @@ struct ChunkArgs {
     float scale;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ uint32_t f32_to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
+
+// Warp-level D += A(16x8, row) * B(8x8, col) in tf32 with fp32 accumulation.
+__device__ __forceinline__ void mma_tf32_16x8x8(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// fp32 [64][64] scratch tiles of the UT transform, XOR-swizzled by row so that
+// the tf32 mma fragment loads and the row-vector stores are bank-conflict free.
+__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + (c ^ ((r & 7) << 2)); }
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output pass from the segment's true start state.
@@ -106,11 +156,16 @@ template <bool kSummary, typename OutT>
 __global__ void __launch_bounds__(256, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                 const ChunkArgs p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = align1024(smem_raw);
+                 const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw;
     const uint32_t sbase = smem_u32(sm);
+    if (sbase & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
+        if (threadIdx.x == 0) report_timeout(15);
+        return;
+    }
 
+    constexpr bool kStageO = sizeof(OutT) == 2;  // bf16 output leaves through TMA stores
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
@@ -119,15 +174,17 @@ __global__ void __launch_bounds__(256, 1)
     if (kSummary && it.g == it.G - 1) return;  // the last segment's map is never needed
 
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC);  // [64]
-    float* sPreOp = sBeta + 64;                                // [128]
-    float* sPreAcc = sPreOp + 128;                             // [128]
-    float* sPost = sPreAcc + 128;                              // [2][128]
+    float* sFrOp = sBeta + 64;                                 // [128] post(prev) * e^{mp}
+    float* sFrAcc = sFrOp + 128;                               // [128] post(prev) * e^{mk}
+    float* sPost = sFrAcc + 128;                               // [2][128] e^{b_C - mk} per chunk
     float* sCarry = sPost + 256;                               // [256]
-    float* sX = sCarry + 256;                                  // [768]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 768);    // qkg, v, mma
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 256);  // qkg, v, mma
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
-    float* sA = reinterpret_cast<float*>(sm + OFF_WN);  // fp32 [64][64] scratch
-    float* sT = reinterpret_cast<float*>(sm + OFF_UT);  // fp32 [64][64] scratch
+    // UT-transform scratch (dead at that point of the chunk): fp32 A and T over the
+    // g tile, per-warp 16x8 products over -W^T.
+    float* sA = reinterpret_cast<float*>(sm + OFF_G);
+    float* sT = reinterpret_cast<float*>(sm + OFF_G + 16384);
+    float* sXw = reinterpret_cast<float*>(sm + OFF_WN);
 
     if (warp == 0) {
         tmem_alloc(sTmem, 512);
@@ -209,6 +266,8 @@ __global__ void __launch_bounds__(256, 1)
 
     uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
     bool aborted = false;
+    float beta_next = 0.f;  // beta of the next chunk's rows, loaded one chunk ahead (tid < 64)
+    if (tid < 64 && nchunks > 0 && t_begin + tid < t_end) beta_next = p.beta[size_t(t_begin + tid) * H + h];
     const uint32_t id_ap = idesc_bf16(128, 64, 1, 1);   // [Kp;Qp] (MN) x Km (MN)
     const uint32_t id_w = idesc_bf16(128, 64, 0, 0);    // Kp^T (K) x (T beta)^T (K)
     const uint32_t id_u = idesc_bf16(128, 64, 1, 0);    // V^T (MN) x (T beta)^T (K)
@@ -223,28 +282,47 @@ __global__ void __launch_bounds__(256, 1)
         const int len = min(kC, t_end - t0);
         const int cur = c & 1, prev = cur ^ 1;
         const int ch = tid & 127, rh = tid >> 7;
+#ifdef KDA_STAGE_TIMING
+        long long ts_ = clock64();
+#endif
 
         // ===== E: cumulative log decay, reference point, gated operands =====
+        if (!kSummary && tid == 0) bulk_wait_read0();  // the O tile over Kp has been read out
         bool ok = mbar_wait(&bars[0], ph_qkg, 1);
         ph_qkg ^= 1;
         if (tid == 0) pend_qkg = false;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        KDA_STAGE(0);
+        if (len < kC) {  // rows past the end of the sequence: g = k = q = 0 (beta = 0 below)
+            for (int e = tid; e < (kC - len) * 32; e += 256) {
+                const int r = len + (e >> 5), w = e & 31;
+                reinterpret_cast<float4*>(sm + OFF_G)[r * 32 + w] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (w < 16) {
+                    const int box = w >> 3, j = w & 7;
+                    st_shared_v4(sbase + OFF_K + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
+                    if (!kSummary) st_shared_v4(sbase + OFF_Q + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
+                }
+            }
+            __syncthreads();
+        }
         const float* sG = reinterpret_cast<const float*>(sm + OFF_G);
         float bl[32];
         {
             float acc = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const int r = rh * 32 + j;
-                const float gv = (r < len) ? fmaxf(sG[r * kD + ch], kGateFloor) : 0.f;
-                acc += gv;
+                acc += fmaxf(sG[(rh * 32 + j) * kD + ch], kGateFloor);
                 bl[j] = acc;
             }
             sCarry[rh * 128 + ch] = acc;
         }
-        if (tid < 64) sBeta[tid] = (tid < len) ? p.beta[size_t(t0 + tid) * H + h] : 0.f;
-        const float b0 = (len > 0) ? fmaxf(sG[ch], kGateFloor) : 0.f;
+        if (tid < 64) sBeta[tid] = beta_next;
+        const float b0 = fmaxf(sG[ch], kGateFloor);
         __syncthreads();
+        if (tid < 64) {  // prefetch the next chunk's beta (one global load per row)
+            const int tn = t0 + kC + tid;
+            beta_next = (c + 1 < nchunks && tn < t_end) ? p.beta[size_t(tn) * H + h] : 0.f;
+        }
         const float bC = sCarry[ch] + sCarry[128 + ch];
         const float carry = rh ? sCarry[ch] : 0.f;
         const bool fast = __syncthreads_and((b0 - bC) <= kRangeMax) != 0;
@@ -259,6 +337,10 @@ __global__ void __launch_bounds__(256, 1)
             const uint8_t* sQb = sm + OFF_Q;
             const uint8_t* sKb = sm + OFF_K;
             const uint32_t box = uint32_t(ch >> 6) * 8192u;
+            const float sc = p.scale;
+            // Kp = k e^{b-mp}, Qp = q e^{b-mp}, Km = k e^{mk-b}; in the factored case
+            // mp = mk = m and both factors come from one product y = (b - m) log2 e.
+            const float y0 = (carry - mp) * kLog2e, y1 = (mk - carry) * kLog2e;
 #pragma unroll
             for (int jj = 0; jj < 32; jj += 8) {
                 uint32_t pk[4], pq[4], pm[4];
@@ -268,13 +350,17 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int j = jj + e + u, r = rh * 32 + j;
-                        const bool valid = r < len;
-                        const float b = bl[j] + carry;
                         const uint32_t off = box + sw128_off(r, ch & 63);
-                        kv[u] = valid ? bf16_at(sKb, off) : 0.f;
-                        qv[u] = (!kSummary && valid) ? bf16_at(sQb, off) * p.scale : 0.f;
-                        e1[u] = __expf(b - mp);
-                        e2[u] = __expf(mk - b);
+                        kv[u] = bf16_at(sKb, off);
+                        qv[u] = kSummary ? 0.f : bf16_at(sQb, off) * sc;
+                        if (fast) {
+                            const float y = fmaf(bl[j], kLog2e, y0);
+                            e1[u] = ex2_approx(y);
+                            e2[u] = ex2_approx(-y);
+                        } else {
+                            e1[u] = ex2_approx(fmaf(bl[j], kLog2e, y0));
+                            e2[u] = ex2_approx(fmaf(bl[j], -kLog2e, y1));
+                        }
                     }
                     pk[e >> 1] = pack_bf16x2(kv[0] * e1[0], kv[1] * e1[1]);
                     pq[e >> 1] = pack_bf16x2(qv[0] * e1[0], qv[1] * e1[1]);
@@ -287,29 +373,67 @@ __global__ void __launch_bounds__(256, 1)
             }
         }
         if (tid < 128) {
-            sPreOp[ch] = __expf(mp);
-            sPreAcc[ch] = __expf(mk);
-            sPost[cur * 128 + ch] = __expf(bC - mk);
+            const float postp = sPost[prev * 128 + ch];
+            sFrOp[ch] = postp * ex2_approx(mp * kLog2e);
+            sFrAcc[ch] = postp * ex2_approx(mk * kLog2e);
+            sPost[cur * 128 + ch] = ex2_approx((bC - mk) * kLog2e);
         }
         fence_async_smem();
         __syncthreads();
+        KDA_STAGE(1);
 
         // ===== A (scaled by beta, strictly lower) and P (lower incl. diagonal) =====
-        if (fast) {
-            if (tid == 0) {
-                tc_fence_after();
+        if (fast && tid == 0) {
+            tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : 16384u, 1024);
-                    const uint64_t b = sdesc_sw128(sbase + OFF_KM + ks * 2048, 8192, 1024);
-                    umma_bf16(tbase + TM_AP, a, b, id_ap, ks > 0);
-                }
-                umma_commit(&bars[2]);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : 16384u, 1024);
+                const uint64_t b = sdesc_sw128(sbase + OFF_KM + ks * 2048, 8192, 1024);
+                umma_bf16(tbase + TM_AP, a, b, id_ap, ks > 0);
             }
+            umma_commit(&bars[2]);
+        }
+        // ===== S frame (needs only the previous chunk's state; overlaps the A/P MMA):
+        //   S <- S * post(prev);  bf16 operand = S * e^{mp};  TMEM = S * e^{mk}
+        {
+            auto frame = [&](uint32_t tcol, uint32_t st_off0, uint32_t st_off1) {
+                float x[64];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) tmem_ld16(tbase + tcol + lane_off + half * 64 + cb * 16, x + cb * 16);
+                tmem_wait_ld();
+                const uint32_t dst = sbase + (half ? st_off1 : st_off0);
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    const int k0 = half * 64 + cb * 16;
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4) {
+                        const float4 fo = *reinterpret_cast<const float4*>(sFrOp + k0 + j);
+                        const float4 fa = *reinterpret_cast<const float4*>(sFrAcc + k0 + j);
+                        float* xx = x + cb * 16 + j;
+                        pk[j >> 1] = pack_bf16x2(xx[0] * fo.x, xx[1] * fo.y);
+                        pk[(j >> 1) + 1] = pack_bf16x2(xx[2] * fo.z, xx[3] * fo.w);
+                        xx[0] *= fa.x;
+                        xx[1] *= fa.y;
+                        xx[2] *= fa.z;
+                        xx[3] *= fa.w;
+                    }
+                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2), pk[0], pk[1], pk[2], pk[3]);
+                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2 + 1), pk[4], pk[5], pk[6], pk[7]);
+                }
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) tmem_st16(tbase + tcol + lane_off + half * 64 + cb * 16, x + cb * 16);
+            };
+            frame(TM_S, OFF_ST, OFF_ST + 16384);
+            if (kSummary) frame(TM_X, XT0, XT1);
+            tmem_wait_st();
+        }
+        if (fast) {
             ok = mbar_wait(&bars[2], ph_mma, 2);
             ph_mma ^= 1;
             tc_fence_after();
             if (__syncthreads_or(!ok)) { aborted = true; break; }
+            KDA_STAGE(2);
             float vals[32];
             tmem_ld16(tbase + TM_AP + lane_off + half * 32, vals);
             tmem_ld16(tbase + TM_AP + lane_off + half * 32 + 16, vals + 16);
@@ -317,9 +441,14 @@ __global__ void __launch_bounds__(256, 1)
             if (vrow < 64) {
                 const float br = sBeta[vrow];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < 32; j += 4) {
                     const int i = half * 32 + j;
-                    sA[vrow * 64 + i] = (i < vrow) ? br * vals[j] : 0.f;
+                    float4 w4;
+                    w4.x = (i + 0 < vrow) ? br * vals[j + 0] : 0.f;
+                    w4.y = (i + 1 < vrow) ? br * vals[j + 1] : 0.f;
+                    w4.z = (i + 2 < vrow) ? br * vals[j + 2] : 0.f;
+                    w4.w = (i + 3 < vrow) ? br * vals[j + 3] : 0.f;
+                    *reinterpret_cast<float4*>(&sA[sidx(vrow, i)]) = w4;
                 }
             } else if (!kSummary) {
                 const int r = vrow - 64;
@@ -340,33 +469,49 @@ __global__ void __launch_bounds__(256, 1)
             const float* sB = reinterpret_cast<const float*>(sm + OFF_G);
             const uint8_t* sQb = sm + OFF_Q;
             const uint8_t* sKb = sm + OFF_K;
-            for (int e = tid; e < 64 * 64; e += 256) sA[e] = 0.f;
-            if (!kSummary)
-                for (int e = tid; e < 512; e += 256) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
-            __syncthreads();
-            for (int pidx = tid; pidx < 64 * 65 / 2; pidx += 256) {
+            constexpr int kPairs = 64 * 65 / 2, kPer = (kPairs + 255) / 256;
+            float ra[kPer], rp[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int pidx = tid + u * 256;
+                ra[u] = rp[u] = 0.f;
+                if (pidx >= kPairs) continue;
                 int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
                 while (r * (r + 1) / 2 > pidx) --r;
                 while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
                 const int i = pidx - r * (r + 1) / 2;
-                float sa = 0.f, sp = 0.f;
                 if (r < len) {
                     for (int cc = 0; cc < kD; ++cc) {
                         const float f = __expf(sB[r * kD + cc] - sB[i * kD + cc]);
                         const uint32_t offr = uint32_t(cc >> 6) * 8192u + sw128_off(r, cc & 63);
                         const uint32_t offi = uint32_t(cc >> 6) * 8192u + sw128_off(i, cc & 63);
                         const float ki = bf16_at(sKb, offi) * f;
-                        sa += bf16_at(sKb, offr) * ki;
-                        if (!kSummary) sp += bf16_at(sQb, offr) * ki;
+                        ra[u] += bf16_at(sKb, offr) * ki;
+                        if (!kSummary) rp[u] += bf16_at(sQb, offr) * ki;
                     }
                 }
-                if (i < r) sA[r * 64 + i] = sBeta[r] * sa;
+            }
+            __syncthreads();  // the q / k tiles are read; sA overlays them
+            for (int e = tid; e < 64 * 64; e += 256) sA[e] = 0.f;
+            if (!kSummary)
+                for (int e = tid; e < 512; e += 256) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int pidx = tid + u * 256;
+                if (pidx >= kPairs) continue;
+                int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
+                while (r * (r + 1) / 2 > pidx) --r;
+                while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
+                const int i = pidx - r * (r + 1) / 2;
+                if (i < r) sA[sidx(r, i)] = sBeta[r] * ra[u];
                 if (!kSummary)
                     *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) =
-                        __float2bfloat16_rn(sp * p.scale);
+                        __float2bfloat16_rn(rp[u] * p.scale);
             }
         }
         __syncthreads();
+        KDA_STAGE(3);
 
         // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
         if (tid < 64) {  // 16x16 diagonal blocks: thread (block I, column jc)
@@ -376,47 +521,72 @@ __global__ void __launch_bounds__(256, 1)
             for (int r = 0; r < 16; ++r) {
                 float s = (r == jc) ? 1.f : 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < r; ++s2) s -= sA[(base + r) * 64 + base + s2] * tcol[s2];
+                for (int s2 = 0; s2 < r; ++s2) s -= sA[sidx(base + r, base + s2)] * tcol[s2];
                 tcol[r] = (r >= jc) ? s : 0.f;
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[(base + r) * 64 + base + jc] = tcol[r];
+            for (int r = 0; r < 16; ++r) sT[sidx(base + r, base + jc)] = tcol[r];
         }
+        KDA_STAGE(15);
         __syncthreads();
+        KDA_STAGE(4);
+        // Off-diagonal 16x16 blocks, one diagonal at a time (d = I - J):
+        //   T_IJ = -T_II X,  X = sum_{K=J}^{I-1} A_IK T_KJ,
+        // on tf32 warp MMAs; warp = (block J, 8-column half of the block).
 #pragma unroll 1
-        for (int d = 1; d <= 3; ++d) {  // blocks (I, J) with I - J = d:  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
-            const int nb = 4 - d;
-            for (int e = tid; e < nb * 256; e += 256) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, i = e & 15;
-                float s = 0.f;
-                for (int kk = 16 * J; kk < 16 * I; ++kk) s += sA[(16 * I + r) * 64 + kk] * sT[kk * 64 + 16 * J + i];
-                sX[e] = s;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += 256) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, i = e & 15;
-                float s = 0.f;
-                for (int j2 = 0; j2 <= r; ++j2) s += sT[(16 * I + r) * 64 + 16 * I + j2] * sX[(J << 8) + j2 * 16 + i];
-                sT[(16 * I + r) * 64 + 16 * J + i] = -s;
+        for (int d = 1; d <= 3; ++d) {
+            if (warp < 2 * (4 - d)) {
+                const int J = warp >> 1, I = J + d, nh = warp & 1;
+                const int gq = lane >> 2, tq = lane & 3;
+                const int col = 16 * J + 8 * nh + gq;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const int ra = 16 * I + gq;
+                for (int kc = 16 * J; kc < 16 * I; kc += 8) {
+                    mma_tf32_16x8x8(acc, f32_to_tf32(sA[sidx(ra, kc + tq)]), f32_to_tf32(sA[sidx(ra + 8, kc + tq)]),
+                                    f32_to_tf32(sA[sidx(ra, kc + tq + 4)]), f32_to_tf32(sA[sidx(ra + 8, kc + tq + 4)]),
+                                    f32_to_tf32(sT[sidx(kc + tq, col)]), f32_to_tf32(sT[sidx(kc + tq + 4, col)]));
+                }
+                float* xs = sXw + warp * 128;  // X as a row-major 16x8 tile
+                xs[gq * 8 + 2 * tq] = acc[0];
+                xs[gq * 8 + 2 * tq + 1] = acc[1];
+                xs[(gq + 8) * 8 + 2 * tq] = acc[2];
+                xs[(gq + 8) * 8 + 2 * tq + 1] = acc[3];
+                __syncwarp();
+                float t2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kc = 0; kc < 16; kc += 8) {
+                    const int cd = 16 * I + kc + tq;
+                    mma_tf32_16x8x8(t2, f32_to_tf32(sT[sidx(ra, cd)]), f32_to_tf32(sT[sidx(ra + 8, cd)]),
+                                    f32_to_tf32(sT[sidx(ra, cd + 4)]), f32_to_tf32(sT[sidx(ra + 8, cd + 4)]),
+                                    f32_to_tf32(xs[(kc + tq) * 8 + gq]), f32_to_tf32(xs[(kc + tq + 4) * 8 + gq]));
+                }
+                const int cw = 16 * J + 8 * nh + 2 * tq;
+                sT[sidx(ra, cw)] = -t2[0];
+                sT[sidx(ra, cw + 1)] = -t2[1];
+                sT[sidx(ra + 8, cw)] = -t2[2];
+                sT[sidx(ra + 8, cw + 1)] = -t2[3];
             }
             __syncthreads();
         }
+        KDA_STAGE(5);
         for (int e = tid; e < 64 * 8; e += 256) {  // (T diag(beta)) as bf16 rows [r][i]
             const int r = e >> 3, j = e & 7;
             uint32_t w[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i0 = 8 * j + 2 * u;
-                w[u] = pack_bf16x2(i0 <= r ? sT[r * 64 + i0] * sBeta[i0] : 0.f,
-                                   i0 + 1 <= r ? sT[r * 64 + i0 + 1] * sBeta[i0 + 1] : 0.f);
+                w[u] = pack_bf16x2(i0 <= r ? sT[sidx(r, i0)] * sBeta[i0] : 0.f,
+                                   i0 + 1 <= r ? sT[sidx(r, i0 + 1)] * sBeta[i0 + 1] : 0.f);
             }
             st_shared_v4(sbase + OFF_TB + sw128_chunk(r, j), w[0], w[1], w[2], w[3]);
         }
+        KDA_STAGE(14);
         fence_async_smem();
         ok = mbar_wait(&bars[1], ph_v, 3);
         ph_v ^= 1;
         if (tid == 0) pend_v = false;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        KDA_STAGE(6);
 
         // ===== W^T = Kp^T (T beta)^T and U^T = V^T (T beta)^T =====
         if (tid == 0) {
@@ -434,38 +604,12 @@ __global__ void __launch_bounds__(256, 1)
             }
         }
 
-        // ===== S frame: S <- S * post(prev) ; operand = S * preop ; TMEM = S * preacc =====
-        {
-            auto frame = [&](uint32_t tcol, uint32_t st_off0, uint32_t st_off1) {
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
-                    const int k0 = half * 64 + cb * 16;
-                    float x[16];
-                    tmem_ld16(tbase + tcol + lane_off + k0, x);
-                    tmem_wait_ld();
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        const float x0 = x[j] * sPost[prev * 128 + k0 + j];
-                        const float x1 = x[j + 1] * sPost[prev * 128 + k0 + j + 1];
-                        pk[j >> 1] = pack_bf16x2(x0 * sPreOp[k0 + j], x1 * sPreOp[k0 + j + 1]);
-                        x[j] = x0 * sPreAcc[k0 + j];
-                        x[j + 1] = x1 * sPreAcc[k0 + j + 1];
-                    }
-                    tmem_st16(tbase + tcol + lane_off + k0, x);
-                    const uint32_t dst = sbase + (half ? st_off1 : st_off0);
-                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2), pk[0], pk[1], pk[2], pk[3]);
-                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2 + 1), pk[4], pk[5], pk[6], pk[7]);
-                }
-            };
-            frame(TM_S, OFF_ST, OFF_ST + 16384);
-            if (kSummary) frame(TM_X, XT0, XT1);
-            tmem_wait_st();
-        }
+        KDA_STAGE(7);
         ok = mbar_wait(&bars[2], ph_mma, 4);
         ph_mma ^= 1;
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        KDA_STAGE(8);
         if (tid == 0 && c + 1 < nchunks) {  // V of this chunk is consumed
             issue_v(c + 1);
             pend_v = true;
@@ -485,6 +629,7 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_before();
         __syncthreads();
 
+        KDA_STAGE(9);
         // ===== U~^T = U^T - S'^T W^T ;  O^T = S'^T Qp  (or U_X~^T = -X'^T W^T) =====
         if (tid == 0) {
             tc_fence_after();
@@ -505,6 +650,7 @@ __global__ void __launch_bounds__(256, 1)
         ph_mma ^= 1;
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        KDA_STAGE(10);
         {  // U~^T (and U_X~^T) -> smem, lane = value channel, 32 tokens per thread
             auto spill = [&](uint32_t tcol, uint32_t dst_off) {
                 float u[32];
@@ -524,6 +670,7 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_before();
         __syncthreads();
 
+        KDA_STAGE(11);
         // ===== O^T += U~^T P^T ;  S^T += U~^T Km  (X^T += U_X~^T Km) =====
         if (tid == 0) {
             tc_fence_after();
@@ -543,21 +690,41 @@ __global__ void __launch_bounds__(256, 1)
         ph_mma ^= 1;
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        KDA_STAGE(12);
 
+        bool staged = false;
         if (!kSummary) {  // O^T -> o[t0 + r, h, v]
             float ov[32];
             tmem_ld16(tbase + TM_O + lane_off + half * 32, ov);
             tmem_ld16(tbase + TM_O + lane_off + half * 32 + 16, ov + 16);
             tmem_wait_ld();
-            OutT* o = static_cast<OutT*>(p.o);
+            if (kStageO && len == kC) {
+                // full chunk: transpose through a swizzled [64 tok][128 v] tile (over Kp,
+                // consumed by now) and write it with one TMA store
+                uint8_t* so = sm + OFF_KP + (vrow >> 6) * 8192;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int r = half * 32 + j;
-                if (r < len) o[(size_t(t0 + r) * H + h) * kD + vrow] = from_f32<OutT>(ov[j]);
+                for (int j = 0; j < 32; ++j)
+                    *reinterpret_cast<__nv_bfloat16*>(so + sw128_off(half * 32 + j, vrow & 63)) =
+                        __float2bfloat16_rn(ov[j]);
+                fence_async_smem();
+                staged = true;
+            } else {
+                OutT* o = static_cast<OutT*>(p.o);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int r = half * 32 + j;
+                    if (r < len) o[(size_t(t0 + r) * H + h) * kD + vrow] = from_f32<OutT>(ov[j]);
+                }
             }
         }
         tc_fence_before();
         __syncthreads();
+        if (staged && tid == 0) {
+            tma_store_3d(&tm_o, sm + OFF_KP, 0, h, t0);
+            tma_store_3d(&tm_o, sm + OFF_KP + 8192, 64, h, t0);
+            bulk_commit();
+        }
+        KDA_STAGE(13);
     }
 
     if (!aborted) {
@@ -591,6 +758,7 @@ __global__ void __launch_bounds__(256, 1)
         if (pend_v) mbar_wait(&bars[1], ph_v, 7);
         mbar_wait(&bars[2], ph_mma, 7);
     }
+    if (!kSummary && tid == 0) bulk_wait0();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
@@ -837,12 +1005,14 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         }
     }
 
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     const long long Tmap = pl.Ttot > 0 ? pl.Ttot : 1;
     if (!make_map(&mq, qb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, Tmap, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        !make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, Tmap, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mo, dtype == KDA_FP32 ? vb : o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "cuTensorMapEncodeTiled failed";
         return KDA_ERR_CUDA;
     }
@@ -867,7 +1037,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
     if (pl.scan) {
         if (set_smem_attr<true, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<true, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+        chunk_kernel<true, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
         if (ev) cudaEventRecord(ev[2], stream);
         combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), 16), 256, 0, stream>>>(
             items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
@@ -878,10 +1048,10 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     }
     if (dtype == KDA_FP32) {
         if (set_smem_attr<false, float>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, float><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+        chunk_kernel<false, float><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
     } else {
         if (set_smem_attr<false, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, a);
+        chunk_kernel<false, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
     }
     if (ev) cudaEventRecord(ev[4], stream);
     const cudaError_t e = cudaGetLastError();
@@ -891,6 +1061,17 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     }
     return KDA_OK;
 }
+
+#ifdef KDA_STAGE_TIMING
+extern "C" int kda_debug_stage_cycles(unsigned long long* out, int reset) {
+    if (cudaMemcpyFromSymbol(out, g_stage_cycles, sizeof(unsigned long long) * 32) != cudaSuccess) return 1;
+    if (reset) {
+        unsigned long long z[32] = {};
+        cudaMemcpyToSymbol(g_stage_cycles, z, sizeof(z));
+    }
+    return 0;
+}
+#endif
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
     return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total;

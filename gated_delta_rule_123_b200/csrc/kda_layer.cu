@@ -181,7 +181,7 @@ static bool gemm_bf16(const void* A, int lda, const void* W, int ldw, void* C, i
 }
 
 struct LayerPlan {
-    int HD, nz;
+    int HD, nz, ldz;  // ldz: row stride of z, padded to 8 elements so every row is 16-byte aligned
     size_t off_z, off_q, off_k, off_v, off_a, off_g, off_beta, off_o, off_lt, off_chunk, chunk_bytes, total;
 };
 constexpr size_t kLtWorkspace = 32u << 20;
@@ -193,9 +193,10 @@ static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nse
     LayerPlan p{};
     p.HD = H * kD;
     p.nz = 3 * p.HD + 2 * rank + H;
+    p.ldz = (p.nz + 7) & ~7;
     size_t off = 0;
     const size_t tokHD = size_t(ntok) * p.HD;
-    p.off_z = off; off = up256l(off + size_t(ntok) * p.nz * 2);
+    p.off_z = off; off = up256l(off + size_t(ntok) * p.ldz * 2);
     p.off_q = off; off = up256l(off + tokHD * 2);
     p.off_k = off; off = up256l(off + tokHD * 2);
     p.off_v = off; off = up256l(off + tokHD * 2);
@@ -233,28 +234,28 @@ int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* c
     float* beta = reinterpret_cast<float*>(b + pl.off_beta);
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(b + pl.off_o);
     void* lt = b + pl.off_lt;
-    const int HD = pl.HD, nz = pl.nz;
+    const int HD = pl.HD, nz = pl.nz, ldz = pl.ldz;
     const __nv_bfloat16* zb = z;
 
-    if (!gemm_bf16(x, D, w->W_in, D, z, nz, ntok, nz, D, lt, kLtWorkspace, stream)) {
+    if (!gemm_bf16(x, D, w->W_in, D, z, ldz, ntok, nz, D, lt, kLtWorkspace, stream)) {
         *why = "cuBLASLt input projection failed";
         return KDA_ERR_CUDA;
     }
     {
         const long long warps = (long long)ntok * H * 3;
         conv_silu_norm_kernel<<<unsigned((warps + 7) / 8), 256, 0, stream>>>(
-            zb, nz, static_cast<const __nv_bfloat16*>(w->conv_w), cu, nseq, ntok, H, q, k, v);
+            zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu, nseq, ntok, H, q, k, v);
     }
-    if (!gemm_bf16(zb + 3 * HD, nz, w->W_aup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
+    if (!gemm_bf16(zb + 3 * HD, ldz, w->W_aup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
         *why = "cuBLASLt alpha up-projection failed";
         return KDA_ERR_CUDA;
     }
-    gates_kernel<<<1184, 256, 0, stream>>>(a, zb, nz, 3 * HD + 2 * R, ntok, H, g, beta);
+    gates_kernel<<<1184, 256, 0, stream>>>(a, zb, ldz, 3 * HD + 2 * R, ntok, H, g, beta);
     const int rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
                                     b + pl.off_chunk, pl.chunk_bytes, stream, why);
     if (rc != KDA_OK) return rc;
     // output gate pre-activation reuses the alpha buffer
-    if (!gemm_bf16(zb + 3 * HD + R, nz, w->W_gup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
+    if (!gemm_bf16(zb + 3 * HD + R, ldz, w->W_gup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
         *why = "cuBLASLt gate up-projection failed";
         return KDA_ERR_CUDA;
     }

@@ -45,7 +45,9 @@ def run_both(kda, inp, scale=1.0, l2=False, heads=None):
         o_got = f64(o)[0]
     s_got = f64(fs)
     assert np.isfinite(o_got).all() and np.isfinite(s_got).all()
-    return rel_l2(o_got, o_ref), rel_l2(s_got, s_ref)
+    eo, es = rel_l2(o_got, o_ref), rel_l2(s_got, s_ref)
+    print(f"rel-L2 o={eo:.3e} state={es:.3e}")
+    return eo, es
 
 
 def test_oracle_sized_fp32(kda):

