@@ -84,21 +84,23 @@ constexpr uint32_t OFF_Q = 0;         // [64 tok][128 c]  (two 64-column boxes, 
 constexpr uint32_t OFF_K = 16384;     // [64 tok][128 c]  (TMA)
 constexpr uint32_t OFF_V = 32768;     // [64 tok][128 v]  (TMA; MN-major A of U^T)
 constexpr uint32_t OFF_G = 49152;     // fp32 [64 tok][128 c] (TMA, no swizzle)
-constexpr uint32_t OFF_KP = 81920;    // [128 c][64 tok]  Kp
-constexpr uint32_t OFF_QP = 98304;    // [128 c][64 tok]  Qp (must follow Kp by 16 KB)
-constexpr uint32_t OFF_KM = 114688;   // [128 c][64 tok]  Km
+constexpr uint32_t OFF_KP = 81920;    // [128 c][64 tok]  Kp  (then the O tile for the TMA store)
+constexpr uint32_t OFF_WN = 98304;    // [128 k][64 tok]  -W^T
+constexpr uint32_t OFF_QP = 114688;   // [128 c][64 tok]  Qp: Kp + 32 KB ([Kp;Qp] stack), -W^T + 16 KB ([-W^T|Qp])
 constexpr uint32_t OFF_TB = 131072;   // [64 r][64 i]     T diag(beta)
 constexpr uint32_t OFF_P = 139264;    // [64 r][64 i]     P (lower incl. diagonal)
-constexpr uint32_t OFF_WN = 147456;   // [128 k][64 tok]  -W^T  (also fp32 A scratch)
-constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S^T (operand copy)
-constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T (also fp32 T scratch)
+constexpr uint32_t OFF_KM = 147456;   // [128 c][64 tok]  Km: right after P ([P|Km] as one N=192 operand)
+constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S'^T (operand copy)
+constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T
 constexpr uint32_t OFF_MISC = 212992;
+static_assert(OFF_QP - OFF_KP == 32768 && OFF_QP - OFF_WN == 16384 && OFF_KM - OFF_P == 8192, "operand stacks");
 constexpr uint32_t MISC_BYTES = 7 * 1024;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES;
 // Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
 
-// TMEM columns (512 allocated): S^T | [A;P] | W^T | U^T | O^T (or U_X^T) | X^T
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_U = 256, TM_O = 320, TM_X = 384;
+// TMEM columns (512 allocated): U^T | O^T (or U_X^T) | S^T | [A;P] | W^T | X^T.
+// [U|O] and [O|S] are contiguous so one N=128 and one N=192 MMA can fill them.
+constexpr uint32_t TM_U = 0, TM_O = 64, TM_S = 128, TM_AP = 256, TM_W = 320, TM_X = 384;
 
 struct ChunkArgs {
     const float* beta;
@@ -135,6 +137,14 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                  "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
                  : "memory");
 }
+// 4-byte asynchronous global->shared copy; src_bytes = 0 writes zero.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -173,8 +183,8 @@ __global__ void __launch_bounds__(256, 1)
     const SegItem it = p.items[item_id];
     if (kSummary && it.g == it.G - 1) return;  // the last segment's map is never needed
 
-    float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC);  // [64]
-    float* sFrOp = sBeta + 64;                                 // [128] post(prev) * e^{mp}
+    float* sBeta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64] beta per chunk parity
+    float* sFrOp = sBeta2 + 128;                               // [128] post(prev) * e^{mp}
     float* sFrAcc = sFrOp + 128;                               // [128] post(prev) * e^{mk}
     float* sPost = sFrAcc + 128;                               // [2][128] e^{b_C - mk} per chunk
     float* sCarry = sPost + 256;                               // [256]
@@ -266,14 +276,20 @@ __global__ void __launch_bounds__(256, 1)
 
     uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
     bool aborted = false;
-    float beta_next = 0.f;  // beta of the next chunk's rows, loaded one chunk ahead (tid < 64)
-    if (tid < 64 && nchunks > 0 && t_begin + tid < t_end) beta_next = p.beta[size_t(t_begin + tid) * H + h];
+    auto fetch_beta = [&](int cc) {  // beta of chunk cc's rows into sBeta2[cc & 1], asynchronously (tid < 64)
+        const int tn = t_begin + cc * kC + tid;
+        const bool valid = cc < nchunks && tn < t_end;
+        cp_async4(sBeta2 + (cc & 1) * 64 + tid, p.beta + (valid ? size_t(tn) * H + h : 0), valid ? 4u : 0u);
+    };
+    if (tid < 64) fetch_beta(0);
     const uint32_t id_ap = idesc_bf16(128, 64, 1, 1);   // [Kp;Qp] (MN) x Km (MN)
     const uint32_t id_w = idesc_bf16(128, 64, 0, 0);    // Kp^T (K) x (T beta)^T (K)
     const uint32_t id_u = idesc_bf16(128, 64, 1, 0);    // V^T (MN) x (T beta)^T (K)
     const uint32_t id_so = idesc_bf16(128, 64, 0, 1);   // S^T (K) x {-W^T, Qp} (MN)
-    const uint32_t id_po = idesc_bf16(128, 64, 0, 0);   // U~^T (K) x P^T (K)
     const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // U~^T (K) x Km (K)
+    const uint32_t id_so2 = idesc_bf16(128, 128, 0, 1); // S'^T (K) x [-W^T | Qp] (MN)
+    const uint32_t id_os = idesc_bf16(128, 192, 0, 0);  // U~^T (K) x [P^T | Km] (K)
+    // Summary pass: X'^T operand halves over the unused q / Qp tiles, U_X~^T over T beta + P.
     const uint32_t XT0 = kSummary ? OFF_Q : 0, XT1 = kSummary ? OFF_QP : 0, UXT = OFF_TB;
 
 #pragma unroll 1
@@ -282,6 +298,7 @@ __global__ void __launch_bounds__(256, 1)
         const int len = min(kC, t_end - t0);
         const int cur = c & 1, prev = cur ^ 1;
         const int ch = tid & 127, rh = tid >> 7;
+        const float* sBeta = sBeta2 + cur * 64;
 #ifdef KDA_STAGE_TIMING
         long long ts_ = clock64();
 #endif
@@ -316,13 +333,12 @@ __global__ void __launch_bounds__(256, 1)
             }
             sCarry[rh * 128 + ch] = acc;
         }
-        if (tid < 64) sBeta[tid] = beta_next;
+        if (tid < 64) {  // this chunk's beta has landed; start the next chunk's
+            cp_async_wait_all();
+            fetch_beta(c + 1);
+        }
         const float b0 = fmaxf(sG[ch], kGateFloor);
         __syncthreads();
-        if (tid < 64) {  // prefetch the next chunk's beta (one global load per row)
-            const int tn = t0 + kC + tid;
-            beta_next = (c + 1 < nchunks && tn < t_end) ? p.beta[size_t(tn) * H + h] : 0.f;
-        }
         const float bC = sCarry[ch] + sCarry[128 + ch];
         const float carry = rh ? sCarry[ch] : 0.f;
         const bool fast = __syncthreads_and((b0 - bC) <= kRangeMax) != 0;
@@ -387,7 +403,7 @@ __global__ void __launch_bounds__(256, 1)
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : 16384u, 1024);
+                const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : OFF_QP - OFF_KP, 1024);
                 const uint64_t b = sdesc_sw128(sbase + OFF_KM + ks * 2048, 8192, 1024);
                 umma_bf16(tbase + TM_AP, a, b, id_ap, ks > 0);
             }
@@ -425,7 +441,15 @@ __global__ void __launch_bounds__(256, 1)
                 for (int cb = 0; cb < 4; ++cb) tmem_st16(tbase + tcol + lane_off + half * 64 + cb * 16, x + cb * 16);
             };
             frame(TM_S, OFF_ST, OFF_ST + 16384);
-            if (kSummary) frame(TM_X, XT0, XT1);
+            if (kSummary) {
+                frame(TM_X, XT0, XT1);
+            } else {  // O^T starts at zero: the merged [U~|O] MMA below accumulates into both halves
+                float z[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) z[j] = 0.f;
+                tmem_st16(tbase + TM_O + lane_off + half * 32, z);
+                tmem_st16(tbase + TM_O + lane_off + half * 32 + 16, z);
+            }
             tmem_wait_st();
         }
         if (fast) {
@@ -636,10 +660,12 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a = sdesc_sw128(sbase + OFF_ST + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                umma_bf16(tbase + TM_U, a, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, 1);
                 if (!kSummary) {
-                    umma_bf16(tbase + TM_O, a, sdesc_sw128(sbase + OFF_QP + ks * 2048, 8192, 1024), id_so, ks > 0);
+                    // [U~ | O] += S'^T [-W^T | Qp]: one N=128 MMA per K step
+                    umma_bf16(tbase + TM_U, a, sdesc_sw128(sbase + OFF_WN + ks * 2048, OFF_QP - OFF_WN, 1024),
+                              id_so2, 1);
                 } else {
+                    umma_bf16(tbase + TM_U, a, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, 1);
                     const uint64_t ax = sdesc_sw128(sbase + ((ks >> 2) ? XT1 : XT0) + (ks & 3) * 32, 16, 1024);
                     umma_bf16(tbase + TM_O, ax, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, ks > 0);
                 }
@@ -677,9 +703,10 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t a = sdesc_sw128(sbase + OFF_UT + ks * 32, 16, 1024);
-                if (!kSummary)
-                    umma_bf16(tbase + TM_O, a, sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024), id_po, 1);
-                umma_bf16(tbase + TM_S, a, sdesc_sw128(sbase + OFF_KM + ks * 32, 16, 1024), id_s, 1);
+                if (!kSummary)  // [O | S] += U~^T [P^T | Km]: one N=192 MMA per K step
+                    umma_bf16(tbase + TM_O, a, sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024), id_os, 1);
+                else
+                    umma_bf16(tbase + TM_S, a, sdesc_sw128(sbase + OFF_KM + ks * 32, 16, 1024), id_s, 1);
                 if (kSummary)
                     umma_bf16(tbase + TM_X, sdesc_sw128(sbase + UXT + ks * 32, 16, 1024),
                               sdesc_sw128(sbase + OFF_KM + ks * 32, 16, 1024), id_s, 1);
@@ -759,6 +786,7 @@ __global__ void __launch_bounds__(256, 1)
         mbar_wait(&bars[2], ph_mma, 7);
     }
     if (!kSummary && tid == 0) bulk_wait0();
+    if (tid < 64) cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
