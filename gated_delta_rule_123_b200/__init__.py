@@ -25,7 +25,7 @@ HEAD_DIM = 128
 SYMBOLS = (
     "kda_status_string", "kda_head_dim", "kda_last_error", "kda_device_status",
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
-    "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events",
+    "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
 )
 
 

@@ -1,0 +1,91 @@
+// kda_chunk_fwd_noalloc: chunked prefill for callers that cannot allocate.
+//
+// Some callers have no way to hand the library a workspace: a plugin hosted by
+// a runtime that owns all device memory and exposes no allocator to it, or a
+// latency-critical serving loop that must not call cudaMalloc (which can
+// synchronise the whole device) in the middle of a step.  This entry point runs
+// exactly the kernels of kda_chunk_fwd, but takes its scratch from a file-scope
+// device array instead of a caller workspace.
+//
+// The array is kNoAllocScratchBytes per GPU, reserved on every device that
+// loads this library and held until the process exits.  Host code cannot pass
+// the array's name to a kernel (on the host it is only a stand-in, not a device
+// address), so the device address is looked up with cudaGetSymbolAddress once
+// per device, with that device current, on the first call made on it.  That
+// first call on a device therefore does a little host-side set-up and should
+// come before any stream capture.  Nothing here calls cudaMalloc, cudaFree or
+// any allocating library routine.
+//
+// All calls share the one array: two calls whose kernels overlap on the GPU
+// (different streams, no ordering between them) race on it and corrupt each
+// other's results.  Calls on one stream, or otherwise ordered, are safe.  The
+// array keeps the last call's contents; the chunk path writes every scratch
+// word it reads (segment table, segment states) before reading it, so nothing
+// needs clearing between calls.
+#include <mutex>
+
+#include "kda_common.cuh"
+
+namespace kda {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
+
+// Device address of g_noalloc_scratch on the current device (looked up once).
+static void* noalloc_scratch(const char** why) {
+    static std::mutex mu;
+    static void* addr[kNoAllocMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+        *why = "no usable current CUDA device";
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            *why = cudaGetErrorString(e);
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace kda
+
+extern "C" int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+extern "C" int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                     const float* initial_state, float* final_state, void* o,
+                                     const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dtype,
+                                     float scale, int l2norm_qk, void* stream) {
+    using namespace kda;
+    if (B < 0 || T < 0 || H < 0 || num_seqs < 0)
+        return kda_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H, dtype,
+                             scale, l2norm_qk, nullptr, 0, stream);  // reports the bad size
+    const size_t need = chunk_workspace_bytes(B, T, H, cu_seqlens ? num_seqs : 0, dtype, l2norm_qk);
+    if (need > kNoAllocScratchBytes) {
+        snprintf(t_last_error, sizeof(t_last_error),
+                 "kda_chunk_fwd_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte static "
+                 "array; use kda_chunk_fwd with a workspace",
+                 need, kNoAllocScratchBytes);
+        return KDA_ERR_UNSUPPORTED;
+    }
+    const char* why = "";
+    void* scratch = noalloc_scratch(&why);
+    if (!scratch) {
+        snprintf(t_last_error, sizeof(t_last_error), "kda_chunk_fwd_noalloc: %s", why);
+        return KDA_ERR_CUDA;
+    }
+    return kda_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H, dtype,
+                         scale, l2norm_qk, scratch, need, stream);
+}

@@ -130,6 +130,31 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
                   void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
+ *
+ * No counterpart on the pages: this is a library convenience.  Some callers
+ * cannot provide a device workspace -- e.g. a plugin inside a runtime that
+ * owns all device memory and gives it no allocator, or a serving loop that
+ * must not call cudaMalloc (which may synchronise the device) mid-step.  This
+ * entry point takes the same arguments as kda_chunk_fwd minus the workspace and
+ * runs the same kernels, with its scratch in a static 64 MiB device array that
+ * every GPU loading the library reserves until the process exits.  It never
+ * allocates.
+ *   - A call needing more scratch than 64 MiB (kda_chunk_fwd_workspace() of the
+ *     same arguments; B=1, H=16, T=65536 bf16 needs about 31 MB) returns
+ *     KDA_ERR_UNSUPPORTED without launching; use kda_chunk_fwd instead.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels can overlap on the GPU
+ *     (e.g. on two unordered streams) race and corrupt each other's results.
+ *     Calls ordered on one stream are safe; nothing needs clearing between them.
+ */
+int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *initial_state, float *final_state, void *o, const int32_t *cu_seqlens,
+                          int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk,
+                          void *stream);
+
+/* ------------------------------------------------------------------------
  * kda_decode_step -- one recurrent step for B sequences (one token each).
  *
  * Residual form, "Kimi Linear: An Expressive, Efficient Attention
