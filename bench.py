@@ -289,7 +289,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        T_s, H_s = 4096, H_PREFILL
+        T_s, H_s = args.T, H_PREFILL  # the whole prefill workload, one step
         dt, cores = cpu_oracle_sample(T_s, H_s)
         cpu = {"value": T_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{T_s} tokens x {H_s} heads of the B=1,H=16,T=65536 prefill ({dt:.1f} s)"}

@@ -162,8 +162,10 @@ constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output pass from the segment's true start state.
+constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
+
 template <bool kSummary, typename OutT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                  const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(256, 1)
 
     constexpr bool kStageO = sizeof(OutT) == 2;  // bf16 output leaves through TMA stores
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;  // TMEM lane quadrant; column quarter
     const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
     if (item_id >= *p.n_items) return;
     const SegItem it = p.items[item_id];
@@ -187,14 +189,15 @@ __global__ void __launch_bounds__(256, 1)
     float* sFrOp = sBeta2 + 128;                               // [128] post(prev) * e^{mp}
     float* sFrAcc = sFrOp + 128;                               // [128] post(prev) * e^{mk}
     float* sPost = sFrAcc + 128;                               // [2][128] e^{b_C - mk} per chunk
-    float* sCarry = sPost + 256;                               // [256]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 256);  // qkg, v, mma
+    float* sCarry = sPost + 256;                               // [4][128] row-quarter sums of g
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 512);  // qkg, v, mma
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
-    // UT-transform scratch (dead at that point of the chunk): fp32 A and T over the
-    // g tile, per-warp 16x8 products over -W^T.
-    float* sA = reinterpret_cast<float*>(sm + OFF_G);
-    float* sT = reinterpret_cast<float*>(sm + OFF_G + 16384);
-    float* sXw = reinterpret_cast<float*>(sm + OFF_WN);
+    // UT-transform scratch, in tiles that are dead from the operand stage until the
+    // W^T spill: fp32 A over U~^T, fp32 T over -W^T, per-warp 16x8 products over T beta.
+    float* sA = reinterpret_cast<float*>(sm + OFF_UT);
+    float* sT = reinterpret_cast<float*>(sm + OFF_WN);
+    float* sXw = reinterpret_cast<float*>(sm + OFF_TB);
+    constexpr int kLoader = 96;  // the thread that issues every TMA load (warp 3, lane 0)
 
     if (warp == 0) {
         tmem_alloc(sTmem, 512);
@@ -240,8 +243,8 @@ __global__ void __launch_bounds__(256, 1)
         tma_load_3d(sm + OFF_V, &tm_v, &bars[1], 0, h, t0);
         tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[1], 64, h, t0);
     };
-    bool pend_qkg = false, pend_v = false;  // meaningful in thread 0 only
-    if (tid == 0 && nchunks > 0) {
+    bool pend_qkg = false, pend_v = false;  // meaningful in the loader thread only
+    if (tid == kLoader && nchunks > 0) {
         issue_qkg(0);
         issue_v(0);
         pend_qkg = pend_v = true;
@@ -259,9 +262,9 @@ __global__ void __launch_bounds__(256, 1)
                 src = p.segS + (size_t(item_id) * H + h) * (kD * kD);
         }
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 0; cb < 2; ++cb) {
             float buf[16];
-            const int k0 = half * 64 + cb * 16;
+            const int k0 = part * 32 + cb * 16;
 #pragma unroll
             for (int j = 0; j < 16; ++j) buf[j] = src ? src[size_t(k0 + j) * kD + vrow] : 0.f;
             tmem_st16(tbase + TM_S + lane_off + k0, buf);
@@ -297,21 +300,20 @@ __global__ void __launch_bounds__(256, 1)
         const int t0 = t_begin + c * kC;
         const int len = min(kC, t_end - t0);
         const int cur = c & 1, prev = cur ^ 1;
-        const int ch = tid & 127, rh = tid >> 7;
+        const int ch = tid & 127, rq = tid >> 7;  // channel; row quarter (16 rows)
         const float* sBeta = sBeta2 + cur * 64;
 #ifdef KDA_STAGE_TIMING
         long long ts_ = clock64();
 #endif
 
         // ===== E: cumulative log decay, reference point, gated operands =====
-        if (!kSummary && tid == 0) bulk_wait_read0();  // the O tile over Kp has been read out
         bool ok = mbar_wait(&bars[0], ph_qkg, 1);
         ph_qkg ^= 1;
-        if (tid == 0) pend_qkg = false;
+        if (tid == kLoader) pend_qkg = false;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(0);
         if (len < kC) {  // rows past the end of the sequence: g = k = q = 0 (beta = 0 below)
-            for (int e = tid; e < (kC - len) * 32; e += 256) {
+            for (int e = tid; e < (kC - len) * 32; e += kThreads) {
                 const int r = len + (e >> 5), w = e & 31;
                 reinterpret_cast<float4*>(sm + OFF_G)[r * 32 + w] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (w < 16) {
@@ -323,15 +325,15 @@ __global__ void __launch_bounds__(256, 1)
             __syncthreads();
         }
         const float* sG = reinterpret_cast<const float*>(sm + OFF_G);
-        float bl[32];
+        float bl[16];
         {
             float acc = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                acc += fmaxf(sG[(rh * 32 + j) * kD + ch], kGateFloor);
+            for (int j = 0; j < 16; ++j) {
+                acc += fmaxf(sG[(rq * 16 + j) * kD + ch], kGateFloor);
                 bl[j] = acc;
             }
-            sCarry[rh * 128 + ch] = acc;
+            sCarry[rq * 128 + ch] = acc;
         }
         if (tid < 64) {  // this chunk's beta has landed; start the next chunk's
             cp_async_wait_all();
@@ -339,15 +341,20 @@ __global__ void __launch_bounds__(256, 1)
         }
         const float b0 = fmaxf(sG[ch], kGateFloor);
         __syncthreads();
-        const float bC = sCarry[ch] + sCarry[128 + ch];
-        const float carry = rh ? sCarry[ch] : 0.f;
+        float carry = 0.f, bC = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float cq = sCarry[q * 128 + ch];
+            carry += (q < rq) ? cq : 0.f;
+            bC += cq;
+        }
         const bool fast = __syncthreads_and((b0 - bC) <= kRangeMax) != 0;
         const float m = 0.5f * (b0 + bC);
         const float mp = fast ? m : 0.f, mk = fast ? m : bC;
         if (!fast) {  // keep b for the exact A / P (g is dead once bl holds it)
             float* sB = reinterpret_cast<float*>(sm + OFF_G);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sB[(rh * 32 + j) * kD + ch] = bl[j] + carry;
+            for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + carry;
         }
         {
             const uint8_t* sQb = sm + OFF_Q;
@@ -358,14 +365,14 @@ __global__ void __launch_bounds__(256, 1)
             // mp = mk = m and both factors come from one product y = (b - m) log2 e.
             const float y0 = (carry - mp) * kLog2e, y1 = (mk - carry) * kLog2e;
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 8) {
+            for (int jj = 0; jj < 16; jj += 8) {
                 uint32_t pk[4], pq[4], pm[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     float kv[2], qv[2], e1[2], e2[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int j = jj + e + u, r = rh * 32 + j;
+                        const int j = jj + e + u, r = rq * 16 + j;
                         const uint32_t off = box + sw128_off(r, ch & 63);
                         kv[u] = bf16_at(sKb, off);
                         qv[u] = kSummary ? 0.f : bf16_at(sQb, off) * sc;
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(256, 1)
                     pq[e >> 1] = pack_bf16x2(qv[0] * e1[0], qv[1] * e1[1]);
                     pm[e >> 1] = pack_bf16x2(kv[0] * e2[0], kv[1] * e2[1]);
                 }
-                const int j8 = (rh * 32 + jj) >> 3;
+                const int j8 = (rq * 16 + jj) >> 3;
                 st_shared_v4(sbase + OFF_KP + sw128_chunk(ch, j8), pk[0], pk[1], pk[2], pk[3]);
                 if (!kSummary) st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), pq[0], pq[1], pq[2], pq[3]);
                 st_shared_v4(sbase + OFF_KM + sw128_chunk(ch, j8), pm[0], pm[1], pm[2], pm[3]);
@@ -397,6 +404,10 @@ __global__ void __launch_bounds__(256, 1)
         fence_async_smem();
         __syncthreads();
         KDA_STAGE(1);
+        if (fast && tid == kLoader && c + 1 < nchunks) {  // q, k, g of this chunk are consumed
+            issue_qkg(c + 1);
+            pend_qkg = true;
+        }
 
         // ===== A (scaled by beta, strictly lower) and P (lower incl. diagonal) =====
         if (fast && tid == 0) {
@@ -413,14 +424,14 @@ __global__ void __launch_bounds__(256, 1)
         //   S <- S * post(prev);  bf16 operand = S * e^{mp};  TMEM = S * e^{mk}
         {
             auto frame = [&](uint32_t tcol, uint32_t st_off0, uint32_t st_off1) {
-                float x[64];
+                float x[32];  // key columns [32 part, 32 part + 32) of this lane
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tmem_ld16(tbase + tcol + lane_off + half * 64 + cb * 16, x + cb * 16);
+                for (int cb = 0; cb < 2; ++cb) tmem_ld16(tbase + tcol + lane_off + part * 32 + cb * 16, x + cb * 16);
                 tmem_wait_ld();
-                const uint32_t dst = sbase + (half ? st_off1 : st_off0);
+                const uint32_t dst = sbase + ((part >> 1) ? st_off1 : st_off0);
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    const int k0 = half * 64 + cb * 16;
+                for (int cb = 0; cb < 2; ++cb) {
+                    const int k0 = part * 32 + cb * 16, ck = (part & 1) * 4 + cb * 2;
                     uint32_t pk[8];
 #pragma unroll
                     for (int j = 0; j < 16; j += 4) {
@@ -434,11 +445,11 @@ __global__ void __launch_bounds__(256, 1)
                         xx[2] *= fa.z;
                         xx[3] *= fa.w;
                     }
-                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2), pk[0], pk[1], pk[2], pk[3]);
-                    st_shared_v4(dst + sw128_chunk(vrow, cb * 2 + 1), pk[4], pk[5], pk[6], pk[7]);
+                    st_shared_v4(dst + sw128_chunk(vrow, ck), pk[0], pk[1], pk[2], pk[3]);
+                    st_shared_v4(dst + sw128_chunk(vrow, ck + 1), pk[4], pk[5], pk[6], pk[7]);
                 }
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tmem_st16(tbase + tcol + lane_off + half * 64 + cb * 16, x + cb * 16);
+                for (int cb = 0; cb < 2; ++cb) tmem_st16(tbase + tcol + lane_off + part * 32 + cb * 16, x + cb * 16);
             };
             frame(TM_S, OFF_ST, OFF_ST + 16384);
             if (kSummary) {
@@ -447,26 +458,25 @@ __global__ void __launch_bounds__(256, 1)
                 float z[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) z[j] = 0.f;
-                tmem_st16(tbase + TM_O + lane_off + half * 32, z);
-                tmem_st16(tbase + TM_O + lane_off + half * 32 + 16, z);
+                tmem_st16(tbase + TM_O + lane_off + part * 16, z);
             }
             tmem_wait_st();
         }
+        if (!kSummary && tid == 0) bulk_wait_read0();  // the previous O tile (over U~^T / sA) is read out
         if (fast) {
             ok = mbar_wait(&bars[2], ph_mma, 2);
             ph_mma ^= 1;
             tc_fence_after();
             if (__syncthreads_or(!ok)) { aborted = true; break; }
             KDA_STAGE(2);
-            float vals[32];
-            tmem_ld16(tbase + TM_AP + lane_off + half * 32, vals);
-            tmem_ld16(tbase + TM_AP + lane_off + half * 32 + 16, vals + 16);
+            float vals[16];  // columns [16 part, 16 part + 16)
+            tmem_ld16(tbase + TM_AP + lane_off + part * 16, vals);
             tmem_wait_ld();
             if (vrow < 64) {
                 const float br = sBeta[vrow];
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const int i = half * 32 + j;
+                for (int j = 0; j < 16; j += 4) {
+                    const int i = part * 16 + j;
                     float4 w4;
                     w4.x = (i + 0 < vrow) ? br * vals[j + 0] : 0.f;
                     w4.y = (i + 1 < vrow) ? br * vals[j + 1] : 0.f;
@@ -477,15 +487,15 @@ __global__ void __launch_bounds__(256, 1)
             } else if (!kSummary) {
                 const int r = vrow - 64;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
+                for (int q4 = 0; q4 < 2; ++q4) {
                     uint32_t w[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int i0 = half * 32 + q4 * 8 + 2 * u;
+                        const int i0 = part * 16 + q4 * 8 + 2 * u;
                         w[u] = pack_bf16x2(i0 <= r ? vals[q4 * 8 + 2 * u] : 0.f,
                                            i0 + 1 <= r ? vals[q4 * 8 + 2 * u + 1] : 0.f);
                     }
-                    st_shared_v4(sbase + OFF_P + sw128_chunk(r, half * 4 + q4), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(sbase + OFF_P + sw128_chunk(r, part * 2 + q4), w[0], w[1], w[2], w[3]);
                 }
             }
         } else {
@@ -493,11 +503,11 @@ __global__ void __launch_bounds__(256, 1)
             const float* sB = reinterpret_cast<const float*>(sm + OFF_G);
             const uint8_t* sQb = sm + OFF_Q;
             const uint8_t* sKb = sm + OFF_K;
-            constexpr int kPairs = 64 * 65 / 2, kPer = (kPairs + 255) / 256;
+            constexpr int kPairs = 64 * 65 / 2, kPer = (kPairs + kThreads - 1) / kThreads;
             float ra[kPer], rp[kPer];
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
-                const int pidx = tid + u * 256;
+                const int pidx = tid + u * kThreads;
                 ra[u] = rp[u] = 0.f;
                 if (pidx >= kPairs) continue;
                 int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
@@ -515,14 +525,18 @@ __global__ void __launch_bounds__(256, 1)
                     }
                 }
             }
-            __syncthreads();  // the q / k tiles are read; sA overlays them
-            for (int e = tid; e < 64 * 64; e += 256) sA[e] = 0.f;
+            __syncthreads();  // the q / k / b tiles are read
+            if (tid == kLoader && c + 1 < nchunks) {
+                issue_qkg(c + 1);
+                pend_qkg = true;
+            }
+            for (int e = tid; e < 64 * 64; e += kThreads) sA[e] = 0.f;
             if (!kSummary)
-                for (int e = tid; e < 512; e += 256) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
+                for (int e = tid; e < 512; e += kThreads) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
             __syncthreads();
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
-                const int pidx = tid + u * 256;
+                const int pidx = tid + u * kThreads;
                 if (pidx >= kPairs) continue;
                 int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
                 while (r * (r + 1) / 2 > pidx) --r;
@@ -538,62 +552,105 @@ __global__ void __launch_bounds__(256, 1)
         KDA_STAGE(3);
 
         // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
-        if (tid < 64) {  // 16x16 diagonal blocks: thread (block I, column jc)
+        if (tid < 64) {
+            // 16x16 diagonal blocks: thread (block I, column jc) solves (I + A_II) t = e_jc
+            // right-looking: once t_r is final, every later row's partial sum is updated, so
+            // the dependent chain is one FMA per row
             const int I = tid >> 4, jc = tid & 15, base = 16 * I;
-            float tcol[16];
+            float ps[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) ps[r] = (r == jc) ? 1.f : 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float s = (r == jc) ? 1.f : 0.f;
+                const float tr = (r >= jc) ? ps[r] : 0.f;
+                ps[r] = tr;
 #pragma unroll
-                for (int s2 = 0; s2 < r; ++s2) s -= sA[sidx(base + r, base + s2)] * tcol[s2];
-                tcol[r] = (r >= jc) ? s : 0.f;
+                for (int r2 = r + 1; r2 < 16; ++r2) ps[r2] -= sA[sidx(base + r2, base + r)] * tr;
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[sidx(base + r, base + jc)] = tcol[r];
+            for (int r = 0; r < 16; ++r) sT[sidx(base + r, base + jc)] = ps[r];
         }
         KDA_STAGE(15);
         __syncthreads();
         KDA_STAGE(4);
-        // Off-diagonal 16x16 blocks, one diagonal at a time (d = I - J):
-        //   T_IJ = -T_II X,  X = sum_{K=J}^{I-1} A_IK T_KJ,
-        // on tf32 warp MMAs; warp = (block J, 8-column half of the block).
-#pragma unroll 1
-        for (int d = 1; d <= 3; ++d) {
-            if (warp < 2 * (4 - d)) {
-                const int J = warp >> 1, I = J + d, nh = warp & 1;
-                const int gq = lane >> 2, tq = lane & 3;
-                const int col = 16 * J + 8 * nh + gq;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                const int ra = 16 * I + gq;
-                for (int kc = 16 * J; kc < 16 * I; kc += 8) {
-                    mma_tf32_16x8x8(acc, f32_to_tf32(sA[sidx(ra, kc + tq)]), f32_to_tf32(sA[sidx(ra + 8, kc + tq)]),
-                                    f32_to_tf32(sA[sidx(ra, kc + tq + 4)]), f32_to_tf32(sA[sidx(ra + 8, kc + tq + 4)]),
+        // Off-diagonal 16x16 blocks on tf32 warp MMAs, in two steps.
+        // Step 1 (32x32 diagonal quadrants): T_10 = -D_1 A_10 D_0, T_32 = -D_3 A_32 D_2.
+        // Step 2 (lower-left quadrant), with E_0 = T[0:32,0:32], E_1 = T[32:64,32:64]:
+        //   X = A[32:64, 0:32] E_0;  T_2J = -D_2 X_top;  T_3J = -(T_32 X_top + D_3 X_bot).
+        // Warp task = (output block, 8-column half).
+        {
+            const int gq = lane >> 2, tq = lane & 3;
+            // acc += sA/sT rows [r0, r0+16) x cols [k0, k0+16) times T rows [k0, k0+16) x col
+            auto mma_at = [&](float* acc, const float* srcA, int r0, int k0, int col) {
+#pragma unroll
+                for (int kc = k0; kc < k0 + 16; kc += 8)
+                    mma_tf32_16x8x8(acc, f32_to_tf32(srcA[sidx(r0 + gq, kc + tq)]),
+                                    f32_to_tf32(srcA[sidx(r0 + gq + 8, kc + tq)]),
+                                    f32_to_tf32(srcA[sidx(r0 + gq, kc + tq + 4)]),
+                                    f32_to_tf32(srcA[sidx(r0 + gq + 8, kc + tq + 4)]),
                                     f32_to_tf32(sT[sidx(kc + tq, col)]), f32_to_tf32(sT[sidx(kc + tq + 4, col)]));
-                }
-                float* xs = sXw + warp * 128;  // X as a row-major 16x8 tile
-                xs[gq * 8 + 2 * tq] = acc[0];
-                xs[gq * 8 + 2 * tq + 1] = acc[1];
-                xs[(gq + 8) * 8 + 2 * tq] = acc[2];
-                xs[(gq + 8) * 8 + 2 * tq + 1] = acc[3];
+            };
+            // acc += sT rows [r0, r0+16) x cols [k0, k0+16) times a 16x8 tile x (row-major)
+            auto mma_tx = [&](float* acc, int r0, int k0, const float* x) {
+#pragma unroll
+                for (int kc = 0; kc < 16; kc += 8)
+                    mma_tf32_16x8x8(acc, f32_to_tf32(sT[sidx(r0 + gq, k0 + kc + tq)]),
+                                    f32_to_tf32(sT[sidx(r0 + gq + 8, k0 + kc + tq)]),
+                                    f32_to_tf32(sT[sidx(r0 + gq, k0 + kc + tq + 4)]),
+                                    f32_to_tf32(sT[sidx(r0 + gq + 8, k0 + kc + tq + 4)]),
+                                    f32_to_tf32(x[(kc + tq) * 8 + gq]), f32_to_tf32(x[(kc + tq + 4) * 8 + gq]));
+            };
+            auto put_x = [&](float* x, const float* acc) {
+                x[gq * 8 + 2 * tq] = acc[0];
+                x[gq * 8 + 2 * tq + 1] = acc[1];
+                x[(gq + 8) * 8 + 2 * tq] = acc[2];
+                x[(gq + 8) * 8 + 2 * tq + 1] = acc[3];
+            };
+            auto put_t = [&](int r0, int c0, const float* acc) {  // T block piece = -acc
+                sT[sidx(r0 + gq, c0 + 2 * tq)] = -acc[0];
+                sT[sidx(r0 + gq, c0 + 2 * tq + 1)] = -acc[1];
+                sT[sidx(r0 + gq + 8, c0 + 2 * tq)] = -acc[2];
+                sT[sidx(r0 + gq + 8, c0 + 2 * tq + 1)] = -acc[3];
+            };
+            float* xs = sXw + warp * 256;  // two 16x8 tiles per warp
+            if (warp < 4) {
+                const int J = (warp >> 1) * 2, I = J + 1, nh = warp & 1, col = 16 * J + 8 * nh + gq;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_at(acc, sA, 16 * I, 16 * J, col);  // X = A_IJ D_J
+                put_x(xs, acc);
                 __syncwarp();
                 float t2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kc = 0; kc < 16; kc += 8) {
-                    const int cd = 16 * I + kc + tq;
-                    mma_tf32_16x8x8(t2, f32_to_tf32(sT[sidx(ra, cd)]), f32_to_tf32(sT[sidx(ra + 8, cd)]),
-                                    f32_to_tf32(sT[sidx(ra, cd + 4)]), f32_to_tf32(sT[sidx(ra + 8, cd + 4)]),
-                                    f32_to_tf32(xs[(kc + tq) * 8 + gq]), f32_to_tf32(xs[(kc + tq + 4) * 8 + gq]));
+                mma_tx(t2, 16 * I, 16 * I, xs);  // D_I X
+                put_t(16 * I, 16 * J + 8 * nh, t2);
+            }
+            __syncthreads();
+            if (warp < 8) {
+                const int I = 2 + (warp >> 2), J = (warp >> 1) & 1, nh = warp & 1;
+                const int col = 16 * J + 8 * nh + gq;
+                float xt[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_at(xt, sA, 32, 16 * J, col);  // A_2J T_JJ ... (rows 32..47)
+                if (J == 0) mma_at(xt, sA, 32, 16, col);  // + A_21 T_10
+                put_x(xs, xt);
+                if (I == 3) {
+                    float xb[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_at(xb, sA, 48, 16 * J, col);
+                    if (J == 0) mma_at(xb, sA, 48, 16, col);
+                    put_x(xs + 128, xb);
                 }
-                const int cw = 16 * J + 8 * nh + 2 * tq;
-                sT[sidx(ra, cw)] = -t2[0];
-                sT[sidx(ra, cw + 1)] = -t2[1];
-                sT[sidx(ra + 8, cw)] = -t2[2];
-                sT[sidx(ra + 8, cw + 1)] = -t2[3];
+                __syncwarp();
+                float t2[4] = {0.f, 0.f, 0.f, 0.f};
+                if (I == 2) {
+                    mma_tx(t2, 32, 32, xs);  // D_2 X_top
+                } else {
+                    mma_tx(t2, 48, 32, xs);        // T_32 X_top
+                    mma_tx(t2, 48, 48, xs + 128);  // + D_3 X_bot
+                }
+                put_t(16 * I, 16 * J + 8 * nh, t2);
             }
             __syncthreads();
         }
         KDA_STAGE(5);
-        for (int e = tid; e < 64 * 8; e += 256) {  // (T diag(beta)) as bf16 rows [r][i]
+        for (int e = tid; e < 64 * 8; e += kThreads) {  // (T diag(beta)) as bf16 rows [r][i]
             const int r = e >> 3, j = e & 7;
             uint32_t w[4];
 #pragma unroll
@@ -608,7 +665,7 @@ __global__ void __launch_bounds__(256, 1)
         fence_async_smem();
         ok = mbar_wait(&bars[1], ph_v, 3);
         ph_v ^= 1;
-        if (tid == 0) pend_v = false;
+        if (tid == kLoader) pend_v = false;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(6);
 
@@ -622,10 +679,6 @@ __global__ void __launch_bounds__(256, 1)
                 umma_bf16(tbase + TM_U, sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), bt, id_u, ks > 0);
             }
             umma_commit(&bars[2]);
-            if (c + 1 < nchunks) {  // q, k, g of this chunk are consumed
-                issue_qkg(c + 1);
-                pend_qkg = true;
-            }
         }
 
         KDA_STAGE(7);
@@ -634,18 +687,17 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(8);
-        if (tid == 0 && c + 1 < nchunks) {  // V of this chunk is consumed
+        if (tid == kLoader && c + 1 < nchunks) {  // V of this chunk is consumed
             issue_v(c + 1);
             pend_v = true;
         }
-        {  // -W^T -> smem (lane = key channel k, 32 tokens per thread)
-            float w[32];
-            tmem_ld16(tbase + TM_W + lane_off + half * 32, w);
-            tmem_ld16(tbase + TM_W + lane_off + half * 32 + 16, w + 16);
+        {  // -W^T -> smem (lane = key channel k, 16 tokens per thread)
+            float w[16];
+            tmem_ld16(tbase + TM_W + lane_off + part * 16, w);
             tmem_wait_ld();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                st_shared_v4(sbase + OFF_WN + sw128_chunk(vrow, half * 4 + q4),
+            for (int q4 = 0; q4 < 2; ++q4)
+                st_shared_v4(sbase + OFF_WN + sw128_chunk(vrow, part * 2 + q4),
                              pack_bf16x2(-w[q4 * 8 + 0], -w[q4 * 8 + 1]), pack_bf16x2(-w[q4 * 8 + 2], -w[q4 * 8 + 3]),
                              pack_bf16x2(-w[q4 * 8 + 4], -w[q4 * 8 + 5]), pack_bf16x2(-w[q4 * 8 + 6], -w[q4 * 8 + 7]));
         }
@@ -677,15 +729,14 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(10);
-        {  // U~^T (and U_X~^T) -> smem, lane = value channel, 32 tokens per thread
+        {  // U~^T (and U_X~^T) -> smem, lane = value channel, 16 tokens per thread
             auto spill = [&](uint32_t tcol, uint32_t dst_off) {
-                float u[32];
-                tmem_ld16(tbase + tcol + lane_off + half * 32, u);
-                tmem_ld16(tbase + tcol + lane_off + half * 32 + 16, u + 16);
+                float u[16];
+                tmem_ld16(tbase + tcol + lane_off + part * 16, u);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    st_shared_v4(sbase + dst_off + sw128_chunk(vrow, half * 4 + q4),
+                for (int q4 = 0; q4 < 2; ++q4)
+                    st_shared_v4(sbase + dst_off + sw128_chunk(vrow, part * 2 + q4),
                                  pack_bf16x2(u[q4 * 8 + 0], u[q4 * 8 + 1]), pack_bf16x2(u[q4 * 8 + 2], u[q4 * 8 + 3]),
                                  pack_bf16x2(u[q4 * 8 + 4], u[q4 * 8 + 5]), pack_bf16x2(u[q4 * 8 + 6], u[q4 * 8 + 7]));
             };
@@ -721,25 +772,24 @@ __global__ void __launch_bounds__(256, 1)
 
         bool staged = false;
         if (!kSummary) {  // O^T -> o[t0 + r, h, v]
-            float ov[32];
-            tmem_ld16(tbase + TM_O + lane_off + half * 32, ov);
-            tmem_ld16(tbase + TM_O + lane_off + half * 32 + 16, ov + 16);
+            float ov[16];  // tokens [16 part, 16 part + 16) of value channel vrow
+            tmem_ld16(tbase + TM_O + lane_off + part * 16, ov);
             tmem_wait_ld();
             if (kStageO && len == kC) {
-                // full chunk: transpose through a swizzled [64 tok][128 v] tile (over Kp,
+                // full chunk: transpose through a swizzled [64 tok][128 v] tile (over U~^T,
                 // consumed by now) and write it with one TMA store
-                uint8_t* so = sm + OFF_KP + (vrow >> 6) * 8192;
+                uint8_t* so = sm + OFF_UT + (vrow >> 6) * 8192;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    *reinterpret_cast<__nv_bfloat16*>(so + sw128_off(half * 32 + j, vrow & 63)) =
+                for (int j = 0; j < 16; ++j)
+                    *reinterpret_cast<__nv_bfloat16*>(so + sw128_off(part * 16 + j, vrow & 63)) =
                         __float2bfloat16_rn(ov[j]);
                 fence_async_smem();
                 staged = true;
             } else {
                 OutT* o = static_cast<OutT*>(p.o);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = half * 32 + j;
+                for (int j = 0; j < 16; ++j) {
+                    const int r = part * 16 + j;
                     if (r < len) o[(size_t(t0 + r) * H + h) * kD + vrow] = from_f32<OutT>(ov[j]);
                 }
             }
@@ -747,8 +797,8 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_before();
         __syncthreads();
         if (staged && tid == 0) {
-            tma_store_3d(&tm_o, sm + OFF_KP, 0, h, t0);
-            tma_store_3d(&tm_o, sm + OFF_KP + 8192, 64, h, t0);
+            tma_store_3d(&tm_o, sm + OFF_UT, 0, h, t0);
+            tma_store_3d(&tm_o, sm + OFF_UT + 8192, 64, h, t0);
             bulk_commit();
         }
         KDA_STAGE(13);
@@ -768,8 +818,8 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         auto store = [&](uint32_t tcol, float* dst) {
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                const int k0 = half * 64 + cb * 16;
+            for (int cb = 0; cb < 2; ++cb) {
+                const int k0 = part * 32 + cb * 16;
                 float x[16];
                 tmem_ld16(tbase + tcol + lane_off + k0, x);
                 tmem_wait_ld();
@@ -778,12 +828,28 @@ __global__ void __launch_bounds__(256, 1)
             }
         };
         if (dstS) store(TM_S, dstS);
-        if (dstX) store(TM_X, dstX);
-    } else if (tid == 0) {
-        // let copies still in flight land before the shared memory is released
-        if (pend_qkg) mbar_wait(&bars[0], ph_qkg, 7);
-        if (pend_v) mbar_wait(&bars[1], ph_v, 7);
-        mbar_wait(&bars[2], ph_mma, 7);
+        if (dstX) {  // X stored transposed, [k'][k] (TMEM lane k' owns a contiguous row), for the combine pass
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                const int k0 = part * 32 + cb * 16;
+                float x[16];
+                tmem_ld16(tbase + TM_X + lane_off + k0, x);
+                tmem_wait_ld();
+                float4* d4 = reinterpret_cast<float4*>(dstX + size_t(vrow) * kD + k0);
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    d4[j >> 2] = make_float4(x[j] * sPost[last * 128 + k0 + j], x[j + 1] * sPost[last * 128 + k0 + j + 1],
+                                             x[j + 2] * sPost[last * 128 + k0 + j + 2],
+                                             x[j + 3] * sPost[last * 128 + k0 + j + 3]);
+            }
+        }
+    } else {
+        // let copies and MMAs still in flight land before shared memory and TMEM are released
+        if (tid == kLoader) {
+            if (pend_qkg) mbar_wait(&bars[0], ph_qkg, 7);
+            if (pend_v) mbar_wait(&bars[1], ph_v, 7);
+        }
+        if (tid == 0) mbar_wait(&bars[2], ph_mma, 7);
     }
     if (!kSummary && tid == 0) bulk_wait0();
     if (tid < 64) cp_async_wait_all();
@@ -837,48 +903,89 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
 }
 
 // ---------------------------------------------------------------- combine
-// Chains the segment maps of one (sequence, head, 8-column slice):
-// S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1.
+// Chains the segment maps of one (sequence, head, 16-column slice):
+// S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1 (segment 0
+// gets the initial state).  X_g^T (64 KB, written transposed by the summary
+// pass) streams into shared memory with 1-D bulk copies, double-buffered; each
+// thread owns a 2 x 4 tile of the slice.
+constexpr int kCombCols = 16;
+constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 64;
+
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const float* init,
-                                                      const float* segN, const float* segX, float* segS, int H) {
+                                                      const float* segN, const float* segXt, float* segS, int H) {
     const int item = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
     if (item >= *n_items) return;
     const SegItem it = items[item];
     if (it.g != 0 || it.G < 2) return;
-    __shared__ float sS[kD][8];
+    extern __shared__ __align__(128) uint8_t csm[];
+    float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
+    float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(csm + 2 * 65536 + kD * kCombCols * 4);  // [2]
     const int tid = threadIdx.x;
-    const int k = tid >> 1, j0 = (tid & 1) * 4;
-    for (int e = tid; e < kD * 8; e += 256) {
-        const int kk = e >> 3, jj = e & 7;
-        const float s0 = init ? init[(size_t(it.seq) * H + h) * (kD * kD) + size_t(kk) * kD + 8 * z + jj] : 0.f;
-        sS[kk][jj] = s0;
-        segS[(size_t(item) * H + h) * (kD * kD) + size_t(kk) * kD + 8 * z + jj] = s0;
+    const int k0 = (tid >> 2) * 2, j0 = (tid & 3) * 4;  // rows k0, k0+1; cols j0..j0+3 of the slice
+    const int c0 = kCombCols * z;
+    const size_t hs = size_t(h) * (kD * kD);
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
     }
     __syncthreads();
-    for (int g = 0; g + 1 < it.G; ++g) {
-        const size_t base = (size_t(item + g) * H + h) * (kD * kD);
-        const float4* Xr = reinterpret_cast<const float4*>(segX + base + size_t(k) * kD);
-        float acc[4];
+    auto fetch = [&](int g) {
+        mbar_arrive_expect_tx(&bar[g & 1], 65536u);
+        bulk_load_1d(sX + (g & 1) * kD * kD, segXt + size_t(item + g) * H * (kD * kD) + hs, 65536u, &bar[g & 1]);
+    };
+    if (tid == 0) fetch(0);
+    for (int e = tid; e < kD * kCombCols; e += 256) {
+        const int kk = e / kCombCols, jj = e % kCombCols;
+        const float s0 = init ? init[size_t(it.seq) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] : 0.f;
+        sS[e] = s0;
+        segS[size_t(item) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] = s0;
+    }
+    __syncthreads();
+    bool ok = true;
+    int fetched = 1, g = 0;  // fetches issued (thread 0) and the step being consumed
+    for (; g + 1 < it.G; ++g) {
+        if (tid == 0 && g + 2 < it.G) {
+            fetch(g + 1);
+            fetched = g + 2;
+        }
+        ok = mbar_wait(&bar[g & 1], uint32_t((g >> 1) & 1), 8);
+        if (__syncthreads_or(!ok)) break;
+        const float* X = sX + (g & 1) * kD * kD;
+        const size_t base = size_t(item + g) * H * (kD * kD) + hs;
+        float acc[2][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = segN[base + size_t(k) * kD + 8 * z + j0 + u];
-#pragma unroll 4
-        for (int k4 = 0; k4 < kD / 4; ++k4) {
-            const float4 x = Xr[k4];
-            const float xs[4] = {x.x, x.y, x.z, x.w};
+        for (int r = 0; r < 2; ++r) {
+            const float4 n4 = *reinterpret_cast<const float4*>(segN + base + size_t(k0 + r) * kD + c0 + j0);
+            acc[r][0] = n4.x; acc[r][1] = n4.y; acc[r][2] = n4.z; acc[r][3] = n4.w;
+        }
+#pragma unroll 8
+        for (int kp = 0; kp < kD; ++kp) {  // acc[k][j] += X[k][kp] S[kp][j] = Xt[kp][k] S[kp][j]
+            const float2 xv = *reinterpret_cast<const float2*>(X + kp * kD + k0);
+            const float4 sv = *reinterpret_cast<const float4*>(sS + kp * kCombCols + j0);
+            acc[0][0] += xv.x * sv.x; acc[0][1] += xv.x * sv.y; acc[0][2] += xv.x * sv.z; acc[0][3] += xv.x * sv.w;
+            acc[1][0] += xv.y * sv.x; acc[1][1] += xv.y * sv.y; acc[1][2] += xv.y * sv.z; acc[1][3] += xv.y * sv.w;
+        }
+        __syncthreads();  // every thread has read sS and this X buffer
+        const size_t out = size_t(item + g + 1) * H * (kD * kD) + hs;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] += xs[w] * sS[4 * k4 + w][j0 + u];
-            }
+        for (int r = 0; r < 2; ++r) {
+            const float4 v4 = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            *reinterpret_cast<float4*>(sS + (k0 + r) * kCombCols + j0) = v4;
+            *reinterpret_cast<float4*>(segS + out + size_t(k0 + r) * kD + c0 + j0) = v4;
         }
         __syncthreads();
-        const size_t out = (size_t(item + g + 1) * H + h) * (kD * kD) + size_t(k) * kD + 8 * z + j0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            sS[k][j0 + u] = acc[u];
-            segS[out + u] = acc[u];
-        }
-        __syncthreads();
+    }
+    if (tid == 0 && !ok) {  // let copies still in flight land before the shared memory is released
+        for (int f = g; f < fetched; ++f) mbar_wait(&bar[f & 1], uint32_t((f >> 1) & 1), 8);
     }
 }
 
@@ -1065,9 +1172,16 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
     if (pl.scan) {
         if (set_smem_attr<true, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<true, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+        chunk_kernel<true, __nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
         if (ev) cudaEventRecord(ev[2], stream);
-        combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), 16), 256, 0, stream>>>(
+        static bool comb_attr = false;
+        if (!comb_attr) {
+            if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombSmem) !=
+                cudaSuccess)
+                return KDA_ERR_CUDA;
+            comb_attr = true;
+        }
+        combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
             items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) cudaEventRecord(ev[3], stream);
     } else if (ev) {
@@ -1076,10 +1190,10 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     }
     if (dtype == KDA_FP32) {
         if (set_smem_attr<false, float>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, float><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+        chunk_kernel<false, float><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
     } else {
         if (set_smem_attr<false, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, __nv_bfloat16><<<grid, 256, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+        chunk_kernel<false, __nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
     }
     if (ev) cudaEventRecord(ev[4], stream);
     const cudaError_t e = cudaGetLastError();
