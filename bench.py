@@ -40,6 +40,21 @@ def metric_name():
         return "KDA prefill tokens/s (H=16,T=64K) + decode state GB/s, % of B200 roofline"
 
 
+def profiled_traffic(summary: str, source: str):
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, or None when the
+    kernel source has changed since the counters were taken (source hash mismatch)."""
+    import hashlib
+    try:
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
+        fields = dict(line.split(":", 1) for line in text.splitlines() if line.startswith(("dram_bytes_per_launch", "kernel_source_sha256")))
+        digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+        if fields.get("kernel_source_sha256", "").strip() != digest:
+            return None
+        return float(fields["dram_bytes_per_launch"].strip())
+    except Exception:
+        return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -218,8 +233,10 @@ def run_ours(args):
     # roofline of the dominant kernel (the output pass): algorithmic bytes per launch / its time
     alg_bytes = BYTES_PER_TOKEN_HEAD * T * H_PREFILL
     achieved = alg_bytes / (out_ms / 1e3) / 1e9
+    traffic = profiled_traffic("chunk_output_T65536_traffic.md", "gated_delta_rule_123_b200/csrc/kda_chunk.cu")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None, "kernel": "chunk_kernel<output>",
+                "frac": achieved / hbm_peak, "traffic": traffic if T == T_PREFILL else None,
+                "traffic_unit": "bytes per launch", "algorithmic_bytes": alg_bytes, "kernel": "chunk_kernel<output>",
                 "peak_kind": peak_kind,
                 "step_frac": alg_bytes / (ms / 1e3) / 1e9 / hbm_peak,
                 "kernel_ms": {"plan": plan_ms, "summary": sum_ms, "combine": comb_ms, "output": out_ms},
