@@ -60,12 +60,12 @@ struct SegItem {
 // Optional per-stage cycle counters (thread 0 of every CTA), compiled in only
 // with -DKDA_STAGE_TIMING for profiling builds.
 #ifdef KDA_STAGE_TIMING
-__device__ unsigned long long g_stage_cycles[32];
+__device__ unsigned long long g_stage_cycles[64];
 #define KDA_STAGE(i)                                                                                   \
     do {                                                                                               \
         if (tid == 0) {                                                                                \
             const long long t_ = clock64();                                                            \
-            atomicAdd(&g_stage_cycles[(kSummary ? 16 : 0) + (i)], (unsigned long long)(t_ - ts_));     \
+            atomicAdd(&g_stage_cycles[(kSummary ? 32 : 0) + (i)], (unsigned long long)(t_ - ts_));     \
             ts_ = t_;                                                                                  \
         }                                                                                              \
     } while (0)
@@ -93,9 +93,11 @@ constexpr uint32_t OFF_KM = 147456;   // [128 c][64 tok]  Km: right after P ([P|
 constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S'^T (operand copy)
 constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T
 constexpr uint32_t OFF_MISC = 212992;
+constexpr uint32_t OFF_XW = OFF_MISC + 7 * 1024;  // 8 KB: per-warp 16x8 products of the UT transform
 static_assert(OFF_QP - OFF_KP == 32768 && OFF_QP - OFF_WN == 16384 && OFF_KM - OFF_P == 8192, "operand stacks");
 constexpr uint32_t MISC_BYTES = 7 * 1024;
-constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES;
+constexpr uint32_t kSmemBytes = OFF_XW + 8192;
+static_assert(OFF_MISC + MISC_BYTES <= OFF_XW && kSmemBytes <= 232448, "shared memory plan");
 // Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
 
 // TMEM columns (512 allocated): U^T | O^T (or U_X^T) | S^T | [A;P] | W^T | X^T.
@@ -160,6 +162,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
+
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output pass from the segment's true start state.
 constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
@@ -193,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 512);  // qkg, v, mma
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
     // UT-transform scratch, in tiles that are dead from the operand stage until the
-    // W^T spill: fp32 A over U~^T, fp32 T over -W^T, per-warp 16x8 products over T beta.
+    // W^T spill: fp32 A over U~^T, fp32 T over -W^T; per-warp 16x8 products in their own tile.
     float* sA = reinterpret_cast<float*>(sm + OFF_UT);
     float* sT = reinterpret_cast<float*>(sm + OFF_WN);
-    float* sXw = reinterpret_cast<float*>(sm + OFF_TB);
+    float* sXw = reinterpret_cast<float*>(sm + OFF_XW);
     constexpr int kLoader = 96;  // the thread that issues every TMA load (warp 3, lane 0)
 
     if (warp == 0) {
@@ -335,12 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             sCarry[rq * 128 + ch] = acc;
         }
+        KDA_STAGE(16);
         if (tid < 64) {  // this chunk's beta has landed; start the next chunk's
             cp_async_wait_all();
             fetch_beta(c + 1);
         }
         const float b0 = fmaxf(sG[ch], kGateFloor);
         __syncthreads();
+        KDA_STAGE(17);
         float carry = 0.f, bC = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -348,21 +353,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             carry += (q < rq) ? cq : 0.f;
             bC += cq;
         }
-        const bool fast = __syncthreads_and((b0 - bC) <= kRangeMax) != 0;
+        const bool fast_here = (b0 - bC) <= kRangeMax;  // this channel's in-chunk decay range
         const float m = 0.5f * (b0 + bC);
-        const float mp = fast ? m : 0.f, mk = fast ? m : bC;
-        if (!fast) {  // keep b for the exact A / P (g is dead once bl holds it)
-            float* sB = reinterpret_cast<float*>(sm + OFF_G);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + carry;
-        }
-        {
+        // Gated operands; factored = the per-channel reference point m (mp = mk = m).
+        // Built speculatively for the factored case; the block-wide vote on the decay
+        // range rides on the stage's closing barrier, and the rare chunk that fails it
+        // is rebuilt with the exact references (mp = 0, mk = b_C).
+        auto emit = [&](const bool factored) {
+            const float mp = factored ? m : 0.f, mk = factored ? m : bC;
             const uint8_t* sQb = sm + OFF_Q;
             const uint8_t* sKb = sm + OFF_K;
             const uint32_t box = uint32_t(ch >> 6) * 8192u;
             const float sc = p.scale;
-            // Kp = k e^{b-mp}, Qp = q e^{b-mp}, Km = k e^{mk-b}; in the factored case
-            // mp = mk = m and both factors come from one product y = (b - m) log2 e.
+            const bool unit_scale = sc == 1.f;
+            // Kp = k e^{b-mp}, Qp = q e^{b-mp}, Km = k e^{mk-b}
             const float y0 = (carry - mp) * kLog2e, y1 = (mk - carry) * kLog2e;
 #pragma unroll
             for (int jj = 0; jj < 16; jj += 8) {
@@ -375,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int j = jj + e + u, r = rq * 16 + j;
                         const uint32_t off = box + sw128_off(r, ch & 63);
                         kv[u] = bf16_at(sKb, off);
-                        qv[u] = kSummary ? 0.f : bf16_at(sQb, off) * sc;
-                        if (fast) {
+                        qv[u] = kSummary ? 0.f : (unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc);
+                        if (factored) {  // one product feeds both factors: y = (b - m) log2 e
                             const float y = fmaf(bl[j], kLog2e, y0);
                             e1[u] = ex2_approx(y);
                             e2[u] = ex2_approx(-y);
@@ -394,15 +398,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!kSummary) st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), pq[0], pq[1], pq[2], pq[3]);
                 st_shared_v4(sbase + OFF_KM + sw128_chunk(ch, j8), pm[0], pm[1], pm[2], pm[3]);
             }
+            if (tid < 128) {
+                const float postp = sPost[prev * 128 + ch];
+                sFrOp[ch] = postp * ex2_approx(mp * kLog2e);
+                sFrAcc[ch] = postp * ex2_approx(mk * kLog2e);
+                sPost[cur * 128 + ch] = ex2_approx((bC - mk) * kLog2e);
+            }
+            fence_async_smem();
+        };
+        KDA_STAGE(18);
+        emit(true);
+        KDA_STAGE(19);
+        const bool fast = __syncthreads_and(fast_here) != 0;
+        if (!fast) {  // exact references; keep b for the exact A / P (g is dead once bl holds it)
+            float* sB = reinterpret_cast<float*>(sm + OFF_G);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + carry;
+            emit(false);
+            __syncthreads();
         }
-        if (tid < 128) {
-            const float postp = sPost[prev * 128 + ch];
-            sFrOp[ch] = postp * ex2_approx(mp * kLog2e);
-            sFrAcc[ch] = postp * ex2_approx(mk * kLog2e);
-            sPost[cur * 128 + ch] = ex2_approx((bC - mk) * kLog2e);
-        }
-        fence_async_smem();
-        __syncthreads();
         KDA_STAGE(1);
         if (fast && tid == kLoader && c + 1 < nchunks) {  // q, k, g of this chunk are consumed
             issue_qkg(c + 1);
@@ -552,11 +566,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         KDA_STAGE(3);
 
         // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
-        if (tid < 64) {
-            // 16x16 diagonal blocks: thread (block I, column jc) solves (I + A_II) t = e_jc
-            // right-looking: once t_r is final, every later row's partial sum is updated, so
-            // the dependent chain is one FMA per row
-            const int I = tid >> 4, jc = tid & 15, base = 16 * I;
+        if (warp < 4 && lane < 16) {
+            // 16x16 diagonal blocks, one per warp on 4 schedulers: lane jc solves
+            // (I + A_II) t = e_jc right-looking: once t_r is final, every later row's
+            // partial sum is updated, so the dependent chain is one FMA per row
+            const int I = warp, jc = lane, base = 16 * I;
             float ps[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) ps[r] = (r == jc) ? 1.f : 0.f;
@@ -567,8 +581,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int r2 = r + 1; r2 < 16; ++r2) ps[r2] -= sA[sidx(base + r2, base + r)] * tr;
             }
+            const float bj = sBeta[base + jc];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[sidx(base + r, base + jc)] = ps[r];
+            for (int r = 0; r < 16; ++r) {
+                sT[sidx(base + r, base + jc)] = ps[r];
+                *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TB + sw128_off(base + r, base + jc)) =
+                    __float2bfloat16_rn(ps[r] * bj);
+            }
+        } else if (tid >= 128 && tid < 128 + 192) {
+            // zero the strictly-upper 16x16 blocks of T beta (16-byte chunks): rows of block I
+            // hold 6 - 2I zero chunks past column 16 (I + 1)
+            const int e = tid - 128, I = e < 96 ? 0 : (e < 160 ? 1 : 2);
+            const int e0 = I == 0 ? e : (I == 1 ? e - 96 : e - 160), per = 6 - 2 * I;
+            const int r = 16 * I + e0 / per, j = 2 * (I + 1) + e0 % per;
+            st_shared_v4(sbase + OFF_TB + sw128_chunk(r, j), 0u, 0u, 0u, 0u);
         }
         KDA_STAGE(15);
         __syncthreads();
@@ -606,11 +632,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 x[(gq + 8) * 8 + 2 * tq] = acc[2];
                 x[(gq + 8) * 8 + 2 * tq + 1] = acc[3];
             };
-            auto put_t = [&](int r0, int c0, const float* acc) {  // T block piece = -acc
-                sT[sidx(r0 + gq, c0 + 2 * tq)] = -acc[0];
-                sT[sidx(r0 + gq, c0 + 2 * tq + 1)] = -acc[1];
-                sT[sidx(r0 + gq + 8, c0 + 2 * tq)] = -acc[2];
-                sT[sidx(r0 + gq + 8, c0 + 2 * tq + 1)] = -acc[3];
+            auto put_t = [&](int r0, int c0, const float* acc) {  // T block piece = -acc (+ bf16 T beta)
+                const int cc = c0 + 2 * tq;
+                sT[sidx(r0 + gq, cc)] = -acc[0];
+                sT[sidx(r0 + gq, cc + 1)] = -acc[1];
+                sT[sidx(r0 + gq + 8, cc)] = -acc[2];
+                sT[sidx(r0 + gq + 8, cc + 1)] = -acc[3];
+                const float b0c = sBeta[cc], b1c = sBeta[cc + 1];
+                *reinterpret_cast<uint32_t*>(sm + OFF_TB + sw128_off(r0 + gq, cc)) =
+                    pack_bf16x2(-acc[0] * b0c, -acc[1] * b1c);
+                *reinterpret_cast<uint32_t*>(sm + OFF_TB + sw128_off(r0 + gq + 8, cc)) =
+                    pack_bf16x2(-acc[2] * b0c, -acc[3] * b1c);
             };
             float* xs = sXw + warp * 256;  // two 16x8 tiles per warp
             if (warp < 4) {
@@ -650,17 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
         KDA_STAGE(5);
-        for (int e = tid; e < 64 * 8; e += kThreads) {  // (T diag(beta)) as bf16 rows [r][i]
-            const int r = e >> 3, j = e & 7;
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i0 = 8 * j + 2 * u;
-                w[u] = pack_bf16x2(i0 <= r ? sT[sidx(r, i0)] * sBeta[i0] : 0.f,
-                                   i0 + 1 <= r ? sT[sidx(r, i0 + 1)] * sBeta[i0 + 1] : 0.f);
-            }
-            st_shared_v4(sbase + OFF_TB + sw128_chunk(r, j), w[0], w[1], w[2], w[3]);
-        }
         KDA_STAGE(14);
         fence_async_smem();
         ok = mbar_wait(&bars[1], ph_v, 3);
@@ -1206,9 +1227,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
 
 #ifdef KDA_STAGE_TIMING
 extern "C" int kda_debug_stage_cycles(unsigned long long* out, int reset) {
-    if (cudaMemcpyFromSymbol(out, g_stage_cycles, sizeof(unsigned long long) * 32) != cudaSuccess) return 1;
+    if (cudaMemcpyFromSymbol(out, g_stage_cycles, sizeof(unsigned long long) * 64) != cudaSuccess) return 1;
     if (reset) {
-        unsigned long long z[32] = {};
+        unsigned long long z[64] = {};
         cudaMemcpyToSymbol(g_stage_cycles, z, sizeof(z));
     }
     return 0;
