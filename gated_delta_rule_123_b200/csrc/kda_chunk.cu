@@ -57,20 +57,29 @@ struct SegItem {
     int pad0, pad1;
 };
 
-// Optional per-stage cycle counters (thread 0 of every CTA), compiled in only
-// with -DKDA_STAGE_TIMING for profiling builds.
+// Optional per-stage cycle counters, compiled in only with -DKDA_STAGE_TIMING for
+// profiling builds.  Thread 0 (stages) and lane 0 of each warp (marks) accumulate
+// in shared memory; each CTA adds its totals to the device arrays once, at exit.
 #ifdef KDA_STAGE_TIMING
 __device__ unsigned long long g_stage_cycles[64];
-#define KDA_STAGE(i)                                                                                   \
-    do {                                                                                               \
-        if (tid == 0) {                                                                                \
-            const long long t_ = clock64();                                                            \
-            atomicAdd(&g_stage_cycles[(kSummary ? 32 : 0) + (i)], (unsigned long long)(t_ - ts_));     \
-            ts_ = t_;                                                                                  \
-        }                                                                                              \
+__device__ unsigned long long g_warp_cycles[2 * 8 * 16];
+#define KDA_STAGE(i)                                  \
+    do {                                              \
+        if (tid == 0) {                               \
+            const long long t_ = clock64();           \
+            s_stage_cyc[(i)] += (unsigned long long)(t_ - ts_); \
+            ts_ = t_;                                 \
+        }                                             \
+    } while (0)
+#define KDA_WMARK(k)                                                                        \
+    do {                                                                                    \
+        if (lane == 0) s_warp_cyc[(k) * 16 + warp] += (unsigned long long)(clock64() - tw0_); \
     } while (0)
 #else
 #define KDA_STAGE(i) \
+    do {             \
+    } while (0)
+#define KDA_WMARK(k) \
     do {             \
     } while (0)
 #endif
@@ -84,20 +93,19 @@ constexpr uint32_t OFF_Q = 0;         // [64 tok][128 c]  (two 64-column boxes, 
 constexpr uint32_t OFF_K = 16384;     // [64 tok][128 c]  (TMA)
 constexpr uint32_t OFF_V = 32768;     // [64 tok][128 v]  (TMA; MN-major A of U^T)
 constexpr uint32_t OFF_G = 49152;     // fp32 [64 tok][128 c] (TMA, no swizzle)
-constexpr uint32_t OFF_KP = 81920;    // [128 c][64 tok]  Kp  (then the O tile for the TMA store)
+constexpr uint32_t OFF_KP = 81920;    // [128 c][64 tok]  Kp
 constexpr uint32_t OFF_WN = 98304;    // [128 k][64 tok]  -W^T
 constexpr uint32_t OFF_QP = 114688;   // [128 c][64 tok]  Qp: Kp + 32 KB ([Kp;Qp] stack), -W^T + 16 KB ([-W^T|Qp])
 constexpr uint32_t OFF_TB = 131072;   // [64 r][64 i]     T diag(beta)
 constexpr uint32_t OFF_P = 139264;    // [64 r][64 i]     P (lower incl. diagonal)
 constexpr uint32_t OFF_KM = 147456;   // [128 c][64 tok]  Km: right after P ([P|Km] as one N=192 operand)
 constexpr uint32_t OFF_ST = 163840;   // 2 x [128 v][64 k] S'^T (operand copy)
-constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T
+constexpr uint32_t OFF_UT = 196608;   // [128 v][64 tok]  U~^T (then the O tile for the TMA store)
 constexpr uint32_t OFF_MISC = 212992;
-constexpr uint32_t OFF_XW = OFF_MISC + 7 * 1024;  // 8 KB: per-warp 16x8 products of the UT transform
 static_assert(OFF_QP - OFF_KP == 32768 && OFF_QP - OFF_WN == 16384 && OFF_KM - OFF_P == 8192, "operand stacks");
 constexpr uint32_t MISC_BYTES = 7 * 1024;
-constexpr uint32_t kSmemBytes = OFF_XW + 8192;
-static_assert(OFF_MISC + MISC_BYTES <= OFF_XW && kSmemBytes <= 232448, "shared memory plan");
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES;
+static_assert(kSmemBytes <= 232448, "shared memory plan");
 // Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
 
 // TMEM columns (512 allocated): U^T | O^T (or U_X^T) | S^T | [A;P] | W^T | X^T.
@@ -118,10 +126,11 @@ struct ChunkArgs {
     float scale;
 };
 
+// fp32 -> tf32 operand, rounded to nearest (ties away from zero) on the integer
+// pipe: add half an ulp of the 10-bit mantissa to the magnitude bits, then drop
+// the 13 low bits.  Finite inputs only.
 __device__ __forceinline__ uint32_t f32_to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
 }
 
 // Warp-level D += A(16x8, row) * B(8x8, col) in tf32 with fp32 accumulation.
@@ -195,11 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sCarry = sPost + 256;                               // [4][128] row-quarter sums of g
     uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 512);  // qkg, v, mma
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
-    // UT-transform scratch, in tiles that are dead from the operand stage until the
-    // W^T spill: fp32 A over U~^T, fp32 T over -W^T; per-warp 16x8 products in their own tile.
+    // UT-transform scratch, in tiles that are dead from the A/P readout until the
+    // W^T spill: fp32 A over U~^T, fp32 T over -W^T.
     float* sA = reinterpret_cast<float*>(sm + OFF_UT);
     float* sT = reinterpret_cast<float*>(sm + OFF_WN);
-    float* sXw = reinterpret_cast<float*>(sm + OFF_XW);
     constexpr int kLoader = 96;  // the thread that issues every TMA load (warp 3, lane 0)
 
     if (warp == 0) {
@@ -219,6 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_g);
     }
     if (tid < 128) sPost[128 + tid] = 1.f;  // the "previous chunk" of chunk 0 scales by 1
+#ifdef KDA_STAGE_TIMING
+    __shared__ unsigned long long s_stage_cyc[32], s_warp_cyc[128];
+    if (tid < 32) s_stage_cyc[tid] = 0;
+    if (tid < 128) s_warp_cyc[tid] = 0;
+#endif
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -298,24 +311,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Summary pass: X'^T operand halves over the unused q / Qp tiles, U_X~^T over T beta + P.
     const uint32_t XT0 = kSummary ? OFF_Q : 0, XT1 = kSummary ? OFF_QP : 0, UXT = OFF_TB;
 
-#pragma unroll 1
-    for (int c = 0; c < nchunks; ++c) {
-        const int t0 = t_begin + c * kC;
-        const int len = min(kC, t_end - t0);
-        const int cur = c & 1, prev = cur ^ 1;
-        const int ch = tid & 127, rq = tid >> 7;  // channel; row quarter (16 rows)
-        const float* sBeta = sBeta2 + cur * 64;
-#ifdef KDA_STAGE_TIMING
-        long long ts_ = clock64();
-#endif
-
-        // ===== E: cumulative log decay, reference point, gated operands =====
-        bool ok = mbar_wait(&bars[0], ph_qkg, 1);
+    // ---- gated operands of a chunk.  Chunk c+1's are built while chunk c's last
+    // tensor-core MMAs run, in pieces placed by which tiles those MMAs still read:
+    //   e_prep : wait for q, k, g; cumulative log decay per channel (registers);
+    //            row-quarter sums to shared memory (a barrier must follow);
+    //   e_head : carry, chunk total b_C, reference point m, this channel's decay range;
+    //   e_rows : factored operands of 8 rows, packed to bf16 in registers;
+    //   e_put_kq / e_put_m : into the Kp, Qp tiles (free once the U~/O MMA is done)
+    //            and the Km tile (free once the O/S MMA is done);
+    //   e_exact: the rare chunk whose decay range failed the vote, rebuilt with the
+    //            exact references (mp = 0, mk = b_C);
+    //   e_frame: per-channel frame factors.
+    const int ch = tid & 127, rq = tid >> 7;  // channel; row quarter (16 rows)
+    const uint32_t e_box = uint32_t(ch >> 6) * 8192u;
+    float bl[16];
+    float e_carry = 0.f, e_bC = 0.f, e_m = 0.f, e_b0 = 0.f;
+    bool e_fast_here = true;
+    uint32_t opk[8], opq[8], opm[8];
+    auto e_prep = [&](int cc) -> bool {  // false: a bounded wait gave up
+        const int len = min(kC, t_end - (t_begin + cc * kC));
+        bool okw = mbar_wait(&bars[0], ph_qkg, 1);
         ph_qkg ^= 1;
         if (tid == kLoader) pend_qkg = false;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        KDA_STAGE(0);
-        if (len < kC) {  // rows past the end of the sequence: g = k = q = 0 (beta = 0 below)
+        if (__syncthreads_or(!okw)) return false;
+        if (len < kC) {  // rows past the end of the sequence: g = k = q = 0 (beta = 0)
             for (int e = tid; e < (kC - len) * 32; e += kThreads) {
                 const int r = len + (e >> 5), w = e & 31;
                 reinterpret_cast<float4*>(sm + OFF_G)[r * 32 + w] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -328,100 +347,155 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
         const float* sG = reinterpret_cast<const float*>(sm + OFF_G);
-        float bl[16];
-        {
-            float acc = 0.f;
+        float acc = 0.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                acc += fmaxf(sG[(rq * 16 + j) * kD + ch], kGateFloor);
-                bl[j] = acc;
-            }
-            sCarry[rq * 128 + ch] = acc;
+        for (int j = 0; j < 16; ++j) {
+            acc += fmaxf(sG[(rq * 16 + j) * kD + ch], kGateFloor);
+            bl[j] = acc;
         }
-        KDA_STAGE(16);
-        if (tid < 64) {  // this chunk's beta has landed; start the next chunk's
+        sCarry[rq * 128 + ch] = acc;
+        e_b0 = fmaxf(sG[ch], kGateFloor);
+        if (tid < 64) {  // this chunk's beta has landed; start the one after it
             cp_async_wait_all();
-            fetch_beta(c + 1);
+            fetch_beta(cc + 1);
         }
-        const float b0 = fmaxf(sG[ch], kGateFloor);
-        __syncthreads();
-        KDA_STAGE(17);
-        float carry = 0.f, bC = 0.f;
+        return true;
+    };
+    auto e_head = [&]() {
+        e_carry = 0.f;
+        e_bC = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float cq = sCarry[q * 128 + ch];
-            carry += (q < rq) ? cq : 0.f;
-            bC += cq;
+            e_carry += (q < rq) ? cq : 0.f;
+            e_bC += cq;
         }
-        const bool fast_here = (b0 - bC) <= kRangeMax;  // this channel's in-chunk decay range
-        const float m = 0.5f * (b0 + bC);
-        // Gated operands; factored = the per-channel reference point m (mp = mk = m).
-        // Built speculatively for the factored case; the block-wide vote on the decay
-        // range rides on the stage's closing barrier, and the rare chunk that fails it
-        // is rebuilt with the exact references (mp = 0, mk = b_C).
-        auto emit = [&](const bool factored) {
-            const float mp = factored ? m : 0.f, mk = factored ? m : bC;
-            const uint8_t* sQb = sm + OFF_Q;
-            const uint8_t* sKb = sm + OFF_K;
-            const uint32_t box = uint32_t(ch >> 6) * 8192u;
-            const float sc = p.scale;
-            const bool unit_scale = sc == 1.f;
-            // Kp = k e^{b-mp}, Qp = q e^{b-mp}, Km = k e^{mk-b}
-            const float y0 = (carry - mp) * kLog2e, y1 = (mk - carry) * kLog2e;
+        e_fast_here = (e_b0 - e_bC) <= kRangeMax;
+        e_m = 0.5f * (e_b0 + e_bC);
+    };
+    // Kp = k e^{b-mp}, Qp = q e^{b-mp}, Km = k e^{mk-b} for rows [8 h8, 8 h8 + 8) of the
+    // quarter; factored (mp = mk = m): one product y = (b - m) log2 e feeds both factors.
+    auto e_rows = [&](const int h8, const bool factored) {
+        const uint8_t* sQb = sm + OFF_Q;
+        const uint8_t* sKb = sm + OFF_K;
+        const float sc = p.scale;
+        const bool unit_scale = sc == 1.f;
+        const float y0 = (factored ? e_carry - e_m : e_carry) * kLog2e;
+        const float y1 = (e_bC - e_carry) * kLog2e;
 #pragma unroll
-            for (int jj = 0; jj < 16; jj += 8) {
-                uint32_t pk[4], pq[4], pm[4];
+        for (int e = 0; e < 8; e += 2) {
+            float kv[2], qv[2], e1[2], e2[2];
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    float kv[2], qv[2], e1[2], e2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int j = jj + e + u, r = rq * 16 + j;
-                        const uint32_t off = box + sw128_off(r, ch & 63);
-                        kv[u] = bf16_at(sKb, off);
-                        qv[u] = kSummary ? 0.f : (unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc);
-                        if (factored) {  // one product feeds both factors: y = (b - m) log2 e
-                            const float y = fmaf(bl[j], kLog2e, y0);
-                            e1[u] = ex2_approx(y);
-                            e2[u] = ex2_approx(-y);
-                        } else {
-                            e1[u] = ex2_approx(fmaf(bl[j], kLog2e, y0));
-                            e2[u] = ex2_approx(fmaf(bl[j], -kLog2e, y1));
-                        }
-                    }
-                    pk[e >> 1] = pack_bf16x2(kv[0] * e1[0], kv[1] * e1[1]);
-                    pq[e >> 1] = pack_bf16x2(qv[0] * e1[0], qv[1] * e1[1]);
-                    pm[e >> 1] = pack_bf16x2(kv[0] * e2[0], kv[1] * e2[1]);
+            for (int u = 0; u < 2; ++u) {
+                const int j = h8 * 8 + e + u, r = rq * 16 + j;
+                const uint32_t off = e_box + sw128_off(r, ch & 63);
+                kv[u] = bf16_at(sKb, off);
+                qv[u] = kSummary ? 0.f : (unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc);
+                if (factored) {
+                    const float y = fmaf(bl[j], kLog2e, y0);
+                    e1[u] = ex2_approx(y);
+                    e2[u] = ex2_approx(-y);
+                } else {
+                    e1[u] = ex2_approx(fmaf(bl[j], kLog2e, y0));
+                    e2[u] = ex2_approx(fmaf(bl[j], -kLog2e, y1));
                 }
-                const int j8 = (rq * 16 + jj) >> 3;
-                st_shared_v4(sbase + OFF_KP + sw128_chunk(ch, j8), pk[0], pk[1], pk[2], pk[3]);
-                if (!kSummary) st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), pq[0], pq[1], pq[2], pq[3]);
-                st_shared_v4(sbase + OFF_KM + sw128_chunk(ch, j8), pm[0], pm[1], pm[2], pm[3]);
             }
-            if (tid < 128) {
-                const float postp = sPost[prev * 128 + ch];
-                sFrOp[ch] = postp * ex2_approx(mp * kLog2e);
-                sFrAcc[ch] = postp * ex2_approx(mk * kLog2e);
-                sPost[cur * 128 + ch] = ex2_approx((bC - mk) * kLog2e);
-            }
-            fence_async_smem();
-        };
-        KDA_STAGE(18);
-        emit(true);
-        KDA_STAGE(19);
-        const bool fast = __syncthreads_and(fast_here) != 0;
-        if (!fast) {  // exact references; keep b for the exact A / P (g is dead once bl holds it)
-            float* sB = reinterpret_cast<float*>(sm + OFF_G);
+            const int slot = h8 * 4 + (e >> 1);
+            opk[slot] = pack_bf16x2(kv[0] * e1[0], kv[1] * e1[1]);
+            opq[slot] = pack_bf16x2(qv[0] * e1[0], qv[1] * e1[1]);
+            opm[slot] = pack_bf16x2(kv[0] * e2[0], kv[1] * e2[1]);
+        }
+    };
+    auto e_put_kq = [&](const int h8) {
+        const int j8 = (rq * 16 + h8 * 8) >> 3;
+        st_shared_v4(sbase + OFF_KP + sw128_chunk(ch, j8), opk[h8 * 4], opk[h8 * 4 + 1], opk[h8 * 4 + 2],
+                     opk[h8 * 4 + 3]);
+        if (!kSummary)
+            st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), opq[h8 * 4], opq[h8 * 4 + 1], opq[h8 * 4 + 2],
+                         opq[h8 * 4 + 3]);
+    };
+    auto e_put_m = [&]() {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + carry;
-            emit(false);
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const int j8 = (rq * 16 + h8 * 8) >> 3;
+            st_shared_v4(sbase + OFF_KM + sw128_chunk(ch, j8), opm[h8 * 4], opm[h8 * 4 + 1], opm[h8 * 4 + 2],
+                         opm[h8 * 4 + 3]);
+        }
+    };
+    // Exact rebuild; the g tile still holds this chunk's gates, so b is recomputed from it
+    // (bl need not stay live) and then kept there for the exact A / P.
+    auto e_exact = [&]() {
+        float* sB = reinterpret_cast<float*>(sm + OFF_G);
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            acc += fmaxf(sB[(rq * 16 + j) * kD + ch], kGateFloor);
+            bl[j] = acc;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + e_carry;
+        e_rows(0, false);
+        e_rows(1, false);
+        e_put_kq(0);
+        e_put_kq(1);
+    };
+    auto e_frame = [&](const int cc, const bool fastc) {
+        if (tid < 128) {
+            const float mp = fastc ? e_m : 0.f, mk = fastc ? e_m : e_bC;
+            const float postp = sPost[((cc & 1) ^ 1) * 128 + ch];
+            sFrOp[ch] = postp * ex2_approx(mp * kLog2e);
+            sFrAcc[ch] = postp * ex2_approx(mk * kLog2e);
+            sPost[(cc & 1) * 128 + ch] = ex2_approx((e_bC - mk) * kLog2e);
+        }
+    };
+
+    // T beta's strictly-upper 16x16 blocks are zeroed every chunk, one 16-byte chunk
+    // per thread < 192: rows of block I hold 6 - 2I zero chunks past column 16 (I + 1).
+    uint32_t tb_zero_addr = 0;
+    if (tid < 192) {
+        const int I = tid < 96 ? 0 : (tid < 160 ? 1 : 2);
+        const int e0 = tid - (I == 0 ? 0 : (I == 1 ? 96 : 160)), per = 6 - 2 * I;
+        tb_zero_addr = sbase + OFF_TB + sw128_chunk(16 * I + e0 / per, 2 * (I + 1) + e0 % per);
+    }
+
+    bool fast_next = true;
+    if (nchunks > 0) {
+        if (!e_prep(0)) {
+            aborted = true;
+        } else {
             __syncthreads();
+            e_head();
+            fast_next = __syncthreads_and(e_fast_here) != 0;
+            if (fast_next) {
+                e_rows(0, true);
+                e_rows(1, true);
+                e_put_kq(0);
+                e_put_kq(1);
+            } else {
+                e_exact();
+            }
+            e_put_m();
+            e_frame(0, fast_next);
+            fence_async_smem();
+            __syncthreads();
+            if (fast_next && tid == kLoader && nchunks > 1) {  // q, k, g of chunk 0 are consumed
+                issue_qkg(1);
+                pend_qkg = true;
+            }
         }
+    }
+
+#pragma unroll 1
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+        const int t0 = t_begin + c * kC;
+        const int len = min(kC, t_end - t0);
+        const float* sBeta = sBeta2 + (c & 1) * 64;
+        const bool fast = fast_next;
+        bool ok = true;
+#ifdef KDA_STAGE_TIMING
+        long long ts_ = clock64(), tw0_ = ts_;
+#endif
         KDA_STAGE(1);
-        if (fast && tid == kLoader && c + 1 < nchunks) {  // q, k, g of this chunk are consumed
-            issue_qkg(c + 1);
-            pend_qkg = true;
-        }
 
         // ===== A (scaled by beta, strictly lower) and P (lower incl. diagonal) =====
         if (fast && tid == 0) {
@@ -483,10 +557,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (__syncthreads_or(!ok)) { aborted = true; break; }
             KDA_STAGE(2);
+#ifdef KDA_STAGE_TIMING
+            tw0_ = clock64();
+#endif
             float vals[16];  // columns [16 part, 16 part + 16)
             tmem_ld16(tbase + TM_AP + lane_off + part * 16, vals);
             tmem_wait_ld();
-            if (vrow < 64) {
+            if (vrow < 64 && part == (vrow >> 4)) {
+                // diagonal 16x16 block of A, stored transposed (A_{r i} at [i][r]) for the
+                // column-per-lane solve below
+                const float br = sBeta[vrow];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int i = part * 16 + j;
+                    sA[sidx(i, vrow)] = (i < vrow) ? br * vals[j] : 0.f;
+                }
+            } else if (vrow < 64) {
                 const float br = sBeta[vrow];
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
@@ -556,83 +642,100 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (r * (r + 1) / 2 > pidx) --r;
                 while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
                 const int i = pidx - r * (r + 1) / 2;
-                if (i < r) sA[sidx(r, i)] = sBeta[r] * ra[u];
+                if (i < r) sA[((r >> 4) == (i >> 4)) ? sidx(i, r) : sidx(r, i)] = sBeta[r] * ra[u];
                 if (!kSummary)
                     *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) =
                         __float2bfloat16_rn(rp[u] * p.scale);
             }
         }
+        KDA_WMARK(0);
         __syncthreads();
+        KDA_WMARK(1);
         KDA_STAGE(3);
 
         // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
         if (warp < 4 && lane < 16) {
-            // 16x16 diagonal blocks, one per warp on 4 schedulers: lane jc solves
-            // (I + A_II) t = e_jc right-looking: once t_r is final, every later row's
-            // partial sum is updated, so the dependent chain is one FMA per row
-            const int I = warp, jc = lane, base = 16 * I;
+            // 16x16 diagonal blocks D_I = (I + A_II)^{-1}: warp I, lane jc solves column jc.
+            // Right-looking: once t_r is final, every later row r2 subtracts A_{r2 r} t_r.
+            // Column r of A_II is row r of the transposed block the readout stored, so
+            // each step reads up to four float4 (the same for all lanes), loaded two
+            // steps ahead so that the chain is one FMA per step.
+            const int base = 16 * warp, jc = lane;
+            const float4* at4 = reinterpret_cast<const float4*>(sA);
+            float4 win[3][4];
+            auto ld_row = [&](float4* dst, const int r) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (4 * q + 3 > r) dst[q] = at4[sidx(base + r, base + 4 * q) >> 2];
+            };
+            ld_row(win[0], 0);
+            ld_row(win[1], 1);
             float ps[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) ps[r] = (r == jc) ? 1.f : 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float tr = (r >= jc) ? ps[r] : 0.f;
-                ps[r] = tr;
+            for (int r = 0; r < 15; ++r) {
+                if (r + 2 < 15) ld_row(win[(r + 2) % 3], r + 2);
+                const float tr = ps[r];
+                const float4* w = win[r % 3];
 #pragma unroll
-                for (int r2 = r + 1; r2 < 16; ++r2) ps[r2] -= sA[sidx(base + r2, base + r)] * tr;
+                for (int q = 0; q < 4; ++q) {
+                    if (4 * q + 0 > r) ps[4 * q + 0] = fmaf(-w[q].x, tr, ps[4 * q + 0]);
+                    if (4 * q + 1 > r) ps[4 * q + 1] = fmaf(-w[q].y, tr, ps[4 * q + 1]);
+                    if (4 * q + 2 > r) ps[4 * q + 2] = fmaf(-w[q].z, tr, ps[4 * q + 2]);
+                    if (4 * q + 3 > r) ps[4 * q + 3] = fmaf(-w[q].w, tr, ps[4 * q + 3]);
+                }
             }
             const float bj = sBeta[base + jc];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 sT[sidx(base + r, base + jc)] = ps[r];
-                *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TB + sw128_off(base + r, base + jc)) =
-                    __float2bfloat16_rn(ps[r] * bj);
+                *reinterpret_cast<uint16_t*>(sm + OFF_TB + sw128_off(base + r, base + jc)) =
+                    uint16_t((__float_as_uint(ps[r] * bj) + 0x8000u) >> 16);
             }
-        } else if (tid >= 128 && tid < 128 + 192) {
-            // zero the strictly-upper 16x16 blocks of T beta (16-byte chunks): rows of block I
-            // hold 6 - 2I zero chunks past column 16 (I + 1)
-            const int e = tid - 128, I = e < 96 ? 0 : (e < 160 ? 1 : 2);
-            const int e0 = I == 0 ? e : (I == 1 ? e - 96 : e - 160), per = 6 - 2 * I;
-            const int r = 16 * I + e0 / per, j = 2 * (I + 1) + e0 % per;
-            st_shared_v4(sbase + OFF_TB + sw128_chunk(r, j), 0u, 0u, 0u, 0u);
         }
+        if (tid < 192) st_shared_v4(tb_zero_addr, 0u, 0u, 0u, 0u);  // strictly-upper blocks of T beta
         KDA_STAGE(15);
+        KDA_WMARK(2);
         __syncthreads();
+        KDA_WMARK(3);
         KDA_STAGE(4);
-        // Off-diagonal 16x16 blocks on tf32 warp MMAs, in two steps.
-        // Step 1 (32x32 diagonal quadrants): T_10 = -D_1 A_10 D_0, T_32 = -D_3 A_32 D_2.
-        // Step 2 (lower-left quadrant), with E_0 = T[0:32,0:32], E_1 = T[32:64,32:64]:
-        //   X = A[32:64, 0:32] E_0;  T_2J = -D_2 X_top;  T_3J = -(T_32 X_top + D_3 X_bot).
+        // Off-diagonal 16x16 blocks on tf32 warp MMAs, each as (L A) R so that the
+        // product L A stays in registers: an accumulator fragment (row g, columns 2t and
+        // 2t+1) is the A operand of the next MMA when the k index is permuted the same
+        // way in the B operand (k slot t <-> row 2t, k slot t+4 <-> row 2t+1).
+        // Level 1: T_IJ = -(D_I A_IJ) D_J for (I, J) = (1,0), (2,1), (3,2).
+        // Level 2 (needs T_10, T_32), with Z_2K = D_2 A_2K and Z_3K = T_32 A_2K + D_3 A_3K:
+        //   T_20 = -(Z_20 D_0 + Z_21 T_10),  T_31 = -Z_31 D_1,  T_30 = -(Z_30 D_0 + Z_31 T_10).
         // Warp task = (output block, 8-column half).
         {
             const int gq = lane >> 2, tq = lane & 3;
-            // acc += sA/sT rows [r0, r0+16) x cols [k0, k0+16) times T rows [k0, k0+16) x col
-            auto mma_at = [&](float* acc, const float* srcA, int r0, int k0, int col) {
+            // y (16x16: fragments for columns [0, 8) and [8, 16)) += L (16x16 at row lr0,
+            // column lk0 of srcL) x R (16x16 at row rk0, column rn0 of srcR)
+            auto mm16 = [&](float* y, const float* srcL, int lr0, int lk0, const float* srcR, int rk0, int rn0) {
 #pragma unroll
-                for (int kc = k0; kc < k0 + 16; kc += 8)
-                    mma_tf32_16x8x8(acc, f32_to_tf32(srcA[sidx(r0 + gq, kc + tq)]),
-                                    f32_to_tf32(srcA[sidx(r0 + gq + 8, kc + tq)]),
-                                    f32_to_tf32(srcA[sidx(r0 + gq, kc + tq + 4)]),
-                                    f32_to_tf32(srcA[sidx(r0 + gq + 8, kc + tq + 4)]),
-                                    f32_to_tf32(sT[sidx(kc + tq, col)]), f32_to_tf32(sT[sidx(kc + tq + 4, col)]));
-            };
-            // acc += sT rows [r0, r0+16) x cols [k0, k0+16) times a 16x8 tile x (row-major)
-            auto mma_tx = [&](float* acc, int r0, int k0, const float* x) {
+                for (int kc = 0; kc < 16; kc += 8) {
+                    const uint32_t a0 = f32_to_tf32(srcL[sidx(lr0 + gq, lk0 + kc + tq)]);
+                    const uint32_t a1 = f32_to_tf32(srcL[sidx(lr0 + gq + 8, lk0 + kc + tq)]);
+                    const uint32_t a2 = f32_to_tf32(srcL[sidx(lr0 + gq, lk0 + kc + tq + 4)]);
+                    const uint32_t a3 = f32_to_tf32(srcL[sidx(lr0 + gq + 8, lk0 + kc + tq + 4)]);
 #pragma unroll
-                for (int kc = 0; kc < 16; kc += 8)
-                    mma_tf32_16x8x8(acc, f32_to_tf32(sT[sidx(r0 + gq, k0 + kc + tq)]),
-                                    f32_to_tf32(sT[sidx(r0 + gq + 8, k0 + kc + tq)]),
-                                    f32_to_tf32(sT[sidx(r0 + gq, k0 + kc + tq + 4)]),
-                                    f32_to_tf32(sT[sidx(r0 + gq + 8, k0 + kc + tq + 4)]),
-                                    f32_to_tf32(x[(kc + tq) * 8 + gq]), f32_to_tf32(x[(kc + tq + 4) * 8 + gq]));
+                    for (int nb = 0; nb < 2; ++nb)
+                        mma_tf32_16x8x8(y + nb * 4, a0, a1, a2, a3,
+                                        f32_to_tf32(srcR[sidx(rk0 + kc + tq, rn0 + nb * 8 + gq)]),
+                                        f32_to_tf32(srcR[sidx(rk0 + kc + tq + 4, rn0 + nb * 8 + gq)]));
+                }
             };
-            auto put_x = [&](float* x, const float* acc) {
-                x[gq * 8 + 2 * tq] = acc[0];
-                x[gq * 8 + 2 * tq + 1] = acc[1];
-                x[(gq + 8) * 8 + 2 * tq] = acc[2];
-                x[(gq + 8) * 8 + 2 * tq + 1] = acc[3];
+            // acc (16x8) += y (16x16, registers) x sT rows [rk0, rk0+16), columns [rn0, rn0+8)
+            auto mm_reg = [&](float* acc, const float* y, int rk0, int rn0) {
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb)
+                    mma_tf32_16x8x8(acc, f32_to_tf32(y[nb * 4 + 0]), f32_to_tf32(y[nb * 4 + 2]),
+                                    f32_to_tf32(y[nb * 4 + 1]), f32_to_tf32(y[nb * 4 + 3]),
+                                    f32_to_tf32(sT[sidx(rk0 + nb * 8 + 2 * tq, rn0 + gq)]),
+                                    f32_to_tf32(sT[sidx(rk0 + nb * 8 + 2 * tq + 1, rn0 + gq)]));
             };
-            auto put_t = [&](int r0, int c0, const float* acc) {  // T block piece = -acc (+ bf16 T beta)
+            auto put_t = [&](int r0, int c0, const float* acc) {  // T block piece = -acc, and its T beta
                 const int cc = c0 + 2 * tq;
                 sT[sidx(r0 + gq, cc)] = -acc[0];
                 sT[sidx(r0 + gq, cc + 1)] = -acc[1];
@@ -644,42 +747,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint32_t*>(sm + OFF_TB + sw128_off(r0 + gq + 8, cc)) =
                     pack_bf16x2(-acc[2] * b0c, -acc[3] * b1c);
             };
-            float* xs = sXw + warp * 256;  // two 16x8 tiles per warp
-            if (warp < 4) {
-                const int J = (warp >> 1) * 2, I = J + 1, nh = warp & 1, col = 16 * J + 8 * nh + gq;
+            if (warp < 6) {
+                const int J = warp >> 1, I = J + 1, cn = 16 * J + 8 * (warp & 1);
+                float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                mm16(y, sT, 16 * I, 16 * I, sA, 16 * I, 16 * J);
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_at(acc, sA, 16 * I, 16 * J, col);  // X = A_IJ D_J
-                put_x(xs, acc);
-                __syncwarp();
-                float t2[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_tx(t2, 16 * I, 16 * I, xs);  // D_I X
-                put_t(16 * I, 16 * J + 8 * nh, t2);
+                mm_reg(acc, y, 16 * J, cn);
+                put_t(16 * I, cn, acc);
             }
+            KDA_WMARK(4);
             __syncthreads();
-            if (warp < 8) {
-                const int I = 2 + (warp >> 2), J = (warp >> 1) & 1, nh = warp & 1;
-                const int col = 16 * J + 8 * nh + gq;
-                float xt[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_at(xt, sA, 32, 16 * J, col);  // A_2J T_JJ ... (rows 32..47)
-                if (J == 0) mma_at(xt, sA, 32, 16, col);  // + A_21 T_10
-                put_x(xs, xt);
-                if (I == 3) {
-                    float xb[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_at(xb, sA, 48, 16 * J, col);
-                    if (J == 0) mma_at(xb, sA, 48, 16, col);
-                    put_x(xs + 128, xb);
+            KDA_WMARK(5);
+            if (warp < 6) {
+                const int task = warp >> 1, cn = 8 * (warp & 1);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                float z0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float z1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                if (task == 0) {  // T_20
+                    mm16(z0, sT, 32, 32, sA, 32, 0);
+                    mm16(z1, sT, 32, 32, sA, 32, 16);
+                    mm_reg(acc, z0, 0, cn);
+                    mm_reg(acc, z1, 16, cn);
+                    put_t(32, cn, acc);
+                } else if (task == 1) {  // T_31
+                    mm16(z1, sT, 48, 32, sA, 32, 16);
+                    mm16(z1, sT, 48, 48, sA, 48, 16);
+                    mm_reg(acc, z1, 16, 16 + cn);
+                    put_t(48, 16 + cn, acc);
+                } else {  // T_30
+                    mm16(z0, sT, 48, 32, sA, 32, 0);
+                    mm16(z1, sT, 48, 32, sA, 32, 16);
+                    mm16(z0, sT, 48, 48, sA, 48, 0);
+                    mm16(z1, sT, 48, 48, sA, 48, 16);
+                    mm_reg(acc, z0, 0, cn);
+                    mm_reg(acc, z1, 16, cn);
+                    put_t(48, cn, acc);
                 }
-                __syncwarp();
-                float t2[4] = {0.f, 0.f, 0.f, 0.f};
-                if (I == 2) {
-                    mma_tx(t2, 32, 32, xs);  // D_2 X_top
-                } else {
-                    mma_tx(t2, 48, 32, xs);        // T_32 X_top
-                    mma_tx(t2, 48, 48, xs + 128);  // + D_3 X_bot
-                }
-                put_t(16 * I, 16 * J + 8 * nh, t2);
             }
+            KDA_WMARK(6);
             __syncthreads();
+            KDA_WMARK(7);
         }
         KDA_STAGE(5);
         KDA_STAGE(14);
@@ -745,11 +852,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma_commit(&bars[2]);
         }
+        // next chunk's operands, first part (the MMA above reads S', -W, Qp)
+        const bool has_next = c + 1 < nchunks;
+        if (has_next) {
+            if (!e_prep(c + 1)) { aborted = true; break; }
+            __syncthreads();  // row-quarter sums
+            e_head();
+            e_rows(0, true);
+        }
+        KDA_STAGE(16);
         ok = mbar_wait(&bars[2], ph_mma, 5);
         ph_mma ^= 1;
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(10);
+        if (has_next) e_put_kq(0);  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
         {  // U~^T (and U_X~^T) -> smem, lane = value channel, 16 tokens per thread
             auto spill = [&](uint32_t tcol, uint32_t dst_off) {
                 float u[16];
@@ -766,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        fast_next = __syncthreads_and(e_fast_here) != 0;  // next chunk's decay-range vote
 
         KDA_STAGE(11);
         // ===== O^T += U~^T P^T ;  S^T += U~^T Km  (X^T += U_X~^T Km) =====
@@ -785,11 +902,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma_commit(&bars[2]);
         }
+        if (has_next && fast_next) {  // second part, overlapping the MMA above (reads U~, P, Km)
+            e_rows(1, true);
+            e_put_kq(1);
+        }
+        KDA_STAGE(18);
         ok = mbar_wait(&bars[2], ph_mma, 6);
         ph_mma ^= 1;
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(12);
+        if (has_next) {  // last part: Km is free now
+            if (!fast_next) e_exact();
+            e_put_m();
+            e_frame(c + 1, fast_next);
+            fence_async_smem();
+        }
+        KDA_STAGE(19);
 
         bool staged = false;
         if (!kSummary) {  // O^T -> o[t0 + r, h, v]
@@ -821,6 +950,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_store_3d(&tm_o, sm + OFF_UT, 0, h, t0);
             tma_store_3d(&tm_o, sm + OFF_UT + 8192, 64, h, t0);
             bulk_commit();
+        }
+        if (has_next && fast_next && tid == kLoader && c + 2 < nchunks) {  // q, k, g of chunk c+1 are consumed
+            issue_qkg(c + 2);
+            pend_qkg = true;
         }
         KDA_STAGE(13);
     }
@@ -876,6 +1009,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < 64) cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
+#ifdef KDA_STAGE_TIMING
+    if (tid < 32) atomicAdd(&g_stage_cycles[(kSummary ? 32 : 0) + tid], s_stage_cyc[tid]);
+    if (tid < 128) atomicAdd(&g_warp_cycles[(kSummary ? 128 : 0) + tid], s_warp_cyc[tid]);
+#endif
     if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
@@ -1231,6 +1368,14 @@ extern "C" int kda_debug_stage_cycles(unsigned long long* out, int reset) {
     if (reset) {
         unsigned long long z[64] = {};
         cudaMemcpyToSymbol(g_stage_cycles, z, sizeof(z));
+    }
+    return 0;
+}
+extern "C" int kda_debug_warp_cycles(unsigned long long* out, int reset) {
+    if (cudaMemcpyFromSymbol(out, g_warp_cycles, sizeof(unsigned long long) * 256) != cudaSuccess) return 1;
+    if (reset) {
+        unsigned long long z[256] = {};
+        cudaMemcpyToSymbol(g_warp_cycles, z, sizeof(z));
     }
     return 0;
 }
