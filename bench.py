@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 T_PREFILL, H_PREFILL, D = 65536, 16, 128
 BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + D * 4 + 4   # q,k,v + o (bf16), g (fp32), beta
+GDN_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + 4 + 4  # q,k,v + o (bf16), one fp32 gate, beta
 FLOP_PER_TOKEN_HEAD = 6 * D * D + 3 * 64 * D + 64 * 64  # the pages' per-head count, C = 64
 
 
@@ -278,6 +279,25 @@ def run_ours(args):
     dec_gbs = dec_bytes / (dec_us / 1e6) / 1e9
     assert kda.device_status() == 0
 
+    # gated DeltaNet fast path on the same workload: one log-gate per (token, head)
+    gs = g[..., 0].contiguous()
+
+    def gstep():
+        kda.gdn_chunk_fwd(q, k, v, gs, beta, initial_state=s0, out=o, final_state=fs, workspace=ws)
+
+    for _ in range(3):
+        gstep()
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        gstep()
+    end.record(stream)
+    torch.cuda.synchronize()
+    gdn_ms = max_over_ranks(start.elapsed_time(end) / args.steps)
+    assert kda.device_status() == 0
+    gdn_bytes = GDN_BYTES_PER_TOKEN_HEAD * T * H_PREFILL
+
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -328,6 +348,10 @@ def run_ours(args):
             "decode": {"workload": "B=256 H=32 d=128, fp32 state in place", "us_per_step": dec_us,
                        "gbs": dec_gbs, "peak_gbs": hbm_peak, "frac": dec_gbs / hbm_peak,
                        "tokens_per_s": world * B / (dec_us / 1e6)},
+            "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
+                    "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
+                    "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,
+                    "step_frac": gdn_bytes / (gdn_ms / 1e3) / 1e9 / hbm_peak},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -26,6 +26,7 @@ SYMBOLS = (
     "kda_status_string", "kda_head_dim", "kda_last_error", "kda_device_status",
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
+    "kda_gdn_chunk_fwd",
 )
 
 
@@ -56,6 +57,8 @@ def _load():
     lib.kda_chunk_fwd_workspace.restype = sz
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i
+    lib.kda_gdn_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.kda_gdn_chunk_fwd.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, f, i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_layer_fwd_workspace.argtypes = [i, i, i, i, i]
@@ -130,6 +133,22 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, scale=1.0, 
 
     q, k, v, g: [B,T,H,128] (or [1,Ttot,H,128] with cu_seqlens); beta: [B,T,H].
     Returns (o, final_state or None)."""
+    return _chunk_call(_lib.kda_chunk_fwd, "kda_chunk_fwd", q, k, v, g, beta, initial_state, cu_seqlens, scale,
+                       l2norm_qk, output_final_state, out, final_state, workspace)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, scale=1.0, l2norm_qk=False,
+                  output_final_state=True, out=None, final_state=None, workspace=None):
+    """Chunkwise prefill with a per-head scalar decay (``kda_gdn_chunk_fwd``).
+
+    q, k, v: [B,T,H,128]; g, beta: [B,T,H] (or [1,Ttot,...] with cu_seqlens).
+    Returns (o, final_state or None)."""
+    return _chunk_call(_lib.kda_gdn_chunk_fwd, "kda_gdn_chunk_fwd", q, k, v, g, beta, initial_state, cu_seqlens,
+                       scale, l2norm_qk, output_final_state, out, final_state, workspace)
+
+
+def _chunk_call(fn, name, q, k, v, g, beta, initial_state, cu_seqlens, scale, l2norm_qk, output_final_state, out,
+                final_state, workspace):
     B, T, H, D = q.shape
     if D != HEAD_DIM:
         raise ValueError("head dim must be 128")
@@ -143,10 +162,10 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, scale=1.0, 
     wsz = chunk_fwd_workspace_bytes(B, T, H, nseq, dt, l2norm_qk)
     if workspace is None or workspace.numel() < wsz:
         workspace = torch.empty(max(wsz, 1), device=q.device, dtype=torch.uint8)
-    rc = _lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(fs), _ptr(o),
-                            _ptr(cu_seqlens), nseq, B, T, H, dt, float(scale), int(l2norm_qk),
-                            _ptr(workspace), wsz, _stream(q.device))
-    _check(rc, "kda_chunk_fwd")
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(fs), _ptr(o),
+            _ptr(cu_seqlens), nseq, B, T, H, dt, float(scale), int(l2norm_qk), _ptr(workspace), wsz,
+            _stream(q.device))
+    _check(rc, name)
     return o, fs
 
 

@@ -12,7 +12,7 @@ int launch_decode_step(const void* q, const void* k, const void* v, const float*
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why);
+                     const char** why, int scalar_gate);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 size_t layer_workspace_bytes(int total_tokens, int d_model, int H, int rank, int num_seqs);
 int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int num_seqs, int total_tokens,
@@ -78,10 +78,12 @@ size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int
     return chunk_workspace_bytes(B, T, H, num_seqs, dtype, l2norm_qk);
 }
 
-int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                  const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens, int num_seqs,
-                  int B, int T, int H, int dtype, float scale, int l2norm_qk, void* workspace,
-                  size_t workspace_bytes, void* stream) {
+// Shared body of kda_chunk_fwd (per-channel g, [.., H, 128]) and kda_gdn_chunk_fwd
+// (one g per token and head, [.., H]).
+static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens,
+                          int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk, void* workspace,
+                          size_t workspace_bytes, void* stream, int scalar_gate) {
     t_last_error[0] = 0;
     if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
     if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
@@ -118,8 +120,24 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     const char* why = "";
     const int rc = launch_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H,
                                     dtype, scale, l2norm_qk, workspace, workspace_bytes,
-                                    static_cast<cudaStream_t>(stream), &why);
+                                    static_cast<cudaStream_t>(stream), &why, scalar_gate);
     return rc == KDA_OK ? KDA_OK : fail(rc, why);
+}
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens, int num_seqs,
+                  int B, int T, int H, int dtype, float scale, int l2norm_qk, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H, dtype,
+                          scale, l2norm_qk, workspace, workspace_bytes, stream, 0);
+}
+
+int kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* initial_state, float* final_state, void* o, const int32_t* cu_seqlens,
+                      int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H, dtype,
+                          scale, l2norm_qk, workspace, workspace_bytes, stream, 1);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,

@@ -114,6 +114,7 @@ constexpr uint32_t TM_U = 0, TM_O = 64, TM_S = 128, TM_AP = 256, TM_W = 320, TM_
 
 struct ChunkArgs {
     const float* beta;
+    const float* gs;  // per-head scalar log-gates [Ttot][H] (scalar-gate kernels only)
     const float* init_state;
     float* final_state;
     void* o;
@@ -174,9 +175,11 @@ constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output pass from the segment's true start state.
+// kScalarGate = true: one log-gate per (token, head) (gated DeltaNet); every key
+// channel shares it, so the decay factors are per row instead of per element.
 constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
 
-template <bool kSummary, typename OutT>
+template <bool kSummary, typename OutT, bool kScalarGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -204,6 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sCarry = sPost + 256;                               // [4][128] row-quarter sums of g
     uint64_t* bars = reinterpret_cast<uint64_t*>(sCarry + 512);  // qkg, v, mma
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+    // scalar gates: [2][64] raw log-gates per chunk parity, and [2][64] per-row
+    // factors e^{b_r - m}, e^{m - b_r} of the chunk being built
+    float* sGs2 = reinterpret_cast<float*>(sm + OFF_MISC + 4864);
+    float* sFac = sGs2 + 128;
     // UT-transform scratch, in tiles that are dead from the A/P readout until the
     // W^T spill: fp32 A over U~^T, fp32 T over -W^T.
     float* sA = reinterpret_cast<float*>(sm + OFF_UT);
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!kSummary) prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        prefetch_tmap(&tm_g);
+        if (!kScalarGate) prefetch_tmap(&tm_g);
     }
     if (tid < 128) sPost[128 + tid] = 1.f;  // the "previous chunk" of chunk 0 scales by 1
 #ifdef KDA_STAGE_TIMING
@@ -244,14 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto issue_qkg = [&](int c) {
         const int t0 = t_begin + c * kC;
-        mbar_arrive_expect_tx(&bars[0], kSummary ? 49152u : 65536u);
+        mbar_arrive_expect_tx(&bars[0], (kSummary ? 49152u : 65536u) - (kScalarGate ? 32768u : 0u));
         if (!kSummary) {
             tma_load_3d(sm + OFF_Q, &tm_q, &bars[0], 0, h, t0);
             tma_load_3d(sm + OFF_Q + 8192, &tm_q, &bars[0], 64, h, t0);
         }
         tma_load_3d(sm + OFF_K, &tm_k, &bars[0], 0, h, t0);
         tma_load_3d(sm + OFF_K + 8192, &tm_k, &bars[0], 64, h, t0);
-        tma_load_3d(sm + OFF_G, &tm_g, &bars[0], 0, h, t0);
+        if (!kScalarGate) tma_load_3d(sm + OFF_G, &tm_g, &bars[0], 0, h, t0);
     };
     auto issue_v = [&](int c) {
         const int t0 = t_begin + c * kC;
@@ -299,6 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tn = t_begin + cc * kC + tid;
         const bool valid = cc < nchunks && tn < t_end;
         cp_async4(sBeta2 + (cc & 1) * 64 + tid, p.beta + (valid ? size_t(tn) * H + h : 0), valid ? 4u : 0u);
+        if (kScalarGate)  // rows past the end read as g = 0
+            cp_async4(sGs2 + (cc & 1) * 64 + tid, p.gs + (valid ? size_t(tn) * H + h : 0), valid ? 4u : 0u);
     };
     if (tid < 64) fetch_beta(0);
     const uint32_t id_ap = idesc_bf16(128, 64, 1, 1);   // [Kp;Qp] (MN) x Km (MN)
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (len < kC) {  // rows past the end of the sequence: g = k = q = 0 (beta = 0)
             for (int e = tid; e < (kC - len) * 32; e += kThreads) {
                 const int r = len + (e >> 5), w = e & 31;
-                reinterpret_cast<float4*>(sm + OFF_G)[r * 32 + w] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (!kScalarGate) reinterpret_cast<float4*>(sm + OFF_G)[r * 32 + w] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (w < 16) {
                     const int box = w >> 3, j = w & 7;
                     st_shared_v4(sbase + OFF_K + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
@@ -345,6 +354,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncthreads();
+        }
+        if (kScalarGate) {
+            if (tid < 64) {  // this chunk's beta and g have landed: inclusive scan of g per warp
+                cp_async_wait_all();
+                float x = fmaxf(sGs2[(cc & 1) * 64 + tid], kGateFloor);
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, d);
+                    if (lane >= d) x += y;
+                }
+                sCarry[tid] = x;  // rows 32..63 still lack rows 0..31's total
+                fetch_beta(cc + 1);
+            }
+            return true;
         }
         const float* sG = reinterpret_cast<const float*>(sm + OFF_G);
         float acc = 0.f;
@@ -361,7 +384,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
     };
+    // scalar gates: b of row r from the per-warp scans (valid between e_prep and the
+    // next chunk's e_prep)
+    auto b_row = [&](int r) { return sCarry[r] + (r >= 32 ? sCarry[31] : 0.f); };
     auto e_head = [&]() {
+        if (kScalarGate) {
+            e_carry = rq ? b_row(rq * 16 - 1) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) bl[j] = b_row(rq * 16 + j) - e_carry;
+            e_b0 = b_row(0);
+            e_bC = b_row(63);
+            e_fast_here = (e_b0 - e_bC) <= kRangeMax;
+            e_m = 0.5f * (e_b0 + e_bC);
+            return;
+        }
         e_carry = 0.f;
         e_bC = 0.f;
 #pragma unroll
@@ -391,7 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t off = e_box + sw128_off(r, ch & 63);
                 kv[u] = bf16_at(sKb, off);
                 qv[u] = kSummary ? 0.f : (unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc);
-                if (factored) {
+                if (factored && kScalarGate) {  // per-row factors, shared by every channel
+                    e1[u] = sFac[r];
+                    e2[u] = sFac[64 + r];
+                } else if (factored) {
                     const float y = fmaf(bl[j], kLog2e, y0);
                     e1[u] = ex2_approx(y);
                     e2[u] = ex2_approx(-y);
@@ -426,11 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (bl need not stay live) and then kept there for the exact A / P.
     auto e_exact = [&]() {
         float* sB = reinterpret_cast<float*>(sm + OFF_G);
-        float acc = 0.f;
+        if (kScalarGate) {  // the g tile is not loaded: b comes from the scans
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            acc += fmaxf(sB[(rq * 16 + j) * kD + ch], kGateFloor);
-            bl[j] = acc;
+            for (int j = 0; j < 16; ++j) bl[j] = b_row(rq * 16 + j) - e_carry;
+        } else {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                acc += fmaxf(sB[(rq * 16 + j) * kD + ch], kGateFloor);
+                bl[j] = acc;
+            }
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) sB[(rq * 16 + j) * kD + ch] = bl[j] + e_carry;
@@ -438,6 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         e_rows(1, false);
         e_put_kq(0);
         e_put_kq(1);
+    };
+    auto e_factors = [&]() {  // scalar gates, factored references: row tid's e^{b-m}, e^{m-b}
+        if (kScalarGate && tid < 64) {
+            const float y = (b_row(tid) - e_m) * kLog2e;
+            sFac[tid] = ex2_approx(y);
+            sFac[64 + tid] = ex2_approx(-y);
+        }
     };
     auto e_frame = [&](const int cc, const bool fastc) {
         if (tid < 128) {
@@ -465,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             __syncthreads();
             e_head();
+            e_factors();
             fast_next = __syncthreads_and(e_fast_here) != 0;
             if (fast_next) {
                 e_rows(0, true);
@@ -856,9 +908,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool has_next = c + 1 < nchunks;
         if (has_next) {
             if (!e_prep(c + 1)) { aborted = true; break; }
-            __syncthreads();  // row-quarter sums
+            __syncthreads();  // row-quarter sums (scalar gates: per-warp scans)
             e_head();
-            e_rows(0, true);
+            if (kScalarGate)
+                e_factors();  // the rows wait for the next barrier
+            else
+                e_rows(0, true);
         }
         KDA_STAGE(16);
         ok = mbar_wait(&bars[2], ph_mma, 5);
@@ -866,7 +921,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(10);
-        if (has_next) e_put_kq(0);  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
+        if (has_next) {  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
+            if (kScalarGate) e_rows(0, true);
+            e_put_kq(0);
+        }
         {  // U~^T (and U_X~^T) -> smem, lane = value channel, 16 tokens per thread
             auto spill = [&](uint32_t tcol, uint32_t dst_off) {
                 float u[16];
@@ -1248,19 +1306,28 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     return pl;
 }
 
-template <bool S, typename O>
+template <bool S, typename O, bool G>
 static cudaError_t set_smem_attr() {
     static bool done = false;
     if (done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(chunk_kernel<S, O>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e =
+        cudaFuncSetAttribute(chunk_kernel<S, O, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess) done = true;
     return e;
+}
+
+template <bool S, typename O, bool G>
+static int launch_pass(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a, cudaStream_t stream) {
+    if (set_smem_attr<S, O, G>() != cudaSuccess) return KDA_ERR_CUDA;
+    chunk_kernel<S, O, G><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+    return KDA_OK;
 }
 
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why) {
+                     const char** why, int scalar_gate) {
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
     if (ws_bytes < pl.total || (pl.total > 0 && ws == nullptr)) {
         *why = "workspace smaller than kda_chunk_fwd_workspace()";
@@ -1303,7 +1370,10 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     if (!make_map(&mq, qb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mk, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mv, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, Tmap, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        // scalar gates are fetched per row, not by TMA: the g map is then a placeholder
+        !make_map(&mg, scalar_gate ? kb : g, scalar_gate ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  scalar_gate ? 2 : 4, H, Tmap, scalar_gate ? 64 : 128,
+                  scalar_gate ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&mo, dtype == KDA_FP32 ? vb : o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "cuTensorMapEncodeTiled failed";
@@ -1317,6 +1387,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
 
     ChunkArgs a{};
     a.beta = beta;
+    a.gs = scalar_gate ? g : nullptr;
     a.init_state = init;
     a.final_state = fin;
     a.o = o;
@@ -1329,8 +1400,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     a.scale = scale;
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
     if (pl.scan) {
-        if (set_smem_attr<true, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<true, __nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+        const int rs = scalar_gate ? launch_pass<true, __nv_bfloat16, true>(grid, mq, mk, mv, mg, mo, a, stream)
+                                   : launch_pass<true, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
+        if (rs != KDA_OK) return rs;
         if (ev) cudaEventRecord(ev[2], stream);
         static bool comb_attr = false;
         if (!comb_attr) {
@@ -1346,13 +1418,14 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         cudaEventRecord(ev[2], stream);
         cudaEventRecord(ev[3], stream);
     }
-    if (dtype == KDA_FP32) {
-        if (set_smem_attr<false, float>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, float><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
-    } else {
-        if (set_smem_attr<false, __nv_bfloat16>() != cudaSuccess) return KDA_ERR_CUDA;
-        chunk_kernel<false, __nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
-    }
+    int ro;
+    if (dtype == KDA_FP32)
+        ro = scalar_gate ? launch_pass<false, float, true>(grid, mq, mk, mv, mg, mo, a, stream)
+                         : launch_pass<false, float, false>(grid, mq, mk, mv, mg, mo, a, stream);
+    else
+        ro = scalar_gate ? launch_pass<false, __nv_bfloat16, true>(grid, mq, mk, mv, mg, mo, a, stream)
+                         : launch_pass<false, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
+    if (ro != KDA_OK) return ro;
     if (ev) cudaEventRecord(ev[4], stream);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

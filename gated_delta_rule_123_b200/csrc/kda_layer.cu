@@ -28,7 +28,7 @@ namespace kda {
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why);
+                     const char** why, int scalar_gate);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 
 __device__ __forceinline__ int seq_start_of(const int32_t* cu, int nseq, int t) {
@@ -252,7 +252,7 @@ int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* c
     }
     gates_kernel<<<1184, 256, 0, stream>>>(a, zb, ldz, 3 * HD + 2 * R, ntok, H, g, beta);
     const int rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
-                                    b + pl.off_chunk, pl.chunk_bytes, stream, why);
+                                    b + pl.off_chunk, pl.chunk_bytes, stream, why, 0);
     if (rc != KDA_OK) return rc;
     // output gate pre-activation reuses the alpha buffer
     if (!gemm_bf16(zb + 3 * HD + R, ldz, w->W_gup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {

@@ -130,6 +130,30 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
                   void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * kda_gdn_chunk_fwd -- chunkwise prefill with a per-head scalar decay (gated
+ * DeltaNet).
+ *
+ * The same recurrence with alpha_t = exp(g_t) * (1, ..., 1): one forgetting
+ * rate per head and token, shared by every key channel.  "Kimi Linear: An
+ * Expressive, Efficient Attention Architecture", section Method, "From Linear
+ * Attention to KDA": GDN adds a per-head scalar forgetting rate; KDA makes it a
+ * per-channel vector.  With g broadcast over the 128 channels, kda_chunk_fwd
+ * computes the same result; this entry point reads 4 bytes of gate per
+ * (token, head) instead of 512 and computes the decay factors once per token
+ * instead of once per (token, channel).
+ *
+ *   g         fp32 [B,T,H] (or [1,Ttot,H] with cu_seqlens): log of the per-head
+ *             decay, expected <= 0 (values below -1e4 are treated as -1e4).
+ *   Every other argument, the layouts, the workspace (size it with
+ *   kda_chunk_fwd_workspace() of the same arguments), the numerics and the
+ *   error behaviour are those of kda_chunk_fwd.
+ */
+int kda_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      const float *initial_state, float *final_state, void *o, const int32_t *cu_seqlens,
+                      int num_seqs, int B, int T, int H, int dtype, float scale, int l2norm_qk,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
  * No counterpart on the pages: this is a library convenience.  Some callers
