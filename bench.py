@@ -279,6 +279,27 @@ def run_ours(args):
     dec_gbs = dec_bytes / (dec_us / 1e6) / 1e9
     assert kda.device_status() == 0
 
+    # fused recurrent segments: 16 tokens per sequence on the decode shape, state in place
+    rT = 16
+    rin = synth.op_inputs(B=B, H=H, T=rT, seed=dcfg["seed"] + 7 + rank, device=dev)
+    orr = torch.empty_like(rin["q"])
+
+    def rstep():
+        kda.recurrent_fwd(rin["q"], rin["k"], rin["v"], rin["g"], rin["beta"], S, out=orr)
+
+    for _ in range(3):
+        rstep()
+    n_rec = 50
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(n_rec):
+        rstep()
+    end.record(stream)
+    torch.cuda.synchronize()
+    rec_us = max_over_ranks(start.elapsed_time(end) / n_rec * 1e3)
+    assert kda.device_status() == 0
+
     # gated DeltaNet fast path on the same workload: one log-gate per (token, head)
     gs = g[..., 0].contiguous()
 
@@ -348,6 +369,9 @@ def run_ours(args):
             "decode": {"workload": "B=256 H=32 d=128, fp32 state in place", "us_per_step": dec_us,
                        "gbs": dec_gbs, "peak_gbs": hbm_peak, "frac": dec_gbs / hbm_peak,
                        "tokens_per_s": world * B / (dec_us / 1e6)},
+            "recurrent": {"workload": f"B={B} H={H} segments of {rT} tokens, fp32 state in place",
+                          "us_per_call": rec_us, "tokens_per_s": world * B * rT / (rec_us / 1e6),
+                          "us_per_token": rec_us / rT},
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,

@@ -26,7 +26,7 @@ SYMBOLS = (
     "kda_status_string", "kda_head_dim", "kda_last_error", "kda_device_status",
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
-    "kda_gdn_chunk_fwd",
+    "kda_gdn_chunk_fwd", "kda_recurrent_fwd",
 )
 
 
@@ -61,6 +61,8 @@ def _load():
     lib.kda_gdn_chunk_fwd.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, f, i, vp]
     lib.kda_decode_step.restype = i
+    lib.kda_recurrent_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.kda_recurrent_fwd.restype = i
     lib.kda_layer_fwd_workspace.argtypes = [i, i, i, i, i]
     lib.kda_layer_fwd_workspace.restype = sz
     lib.kda_layer_fwd.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, i, i, vp, vp, vp, vp, sz, vp]
@@ -178,6 +180,19 @@ def decode_step(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None):
     rc = _lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o), B, H,
                               _dtype_code(q), float(scale), int(l2norm_qk), _stream(q.device))
     _check(rc, "kda_decode_step")
+    return o
+
+
+def recurrent_fwd(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None):
+    """Fused recurrent segment (``kda_recurrent_fwd``): q, k, v, g [B,T,H,128], beta [B,T,H];
+    ``state`` [B,H,128,128] fp32 is updated in place.  Returns o [B,T,H,128]."""
+    B, T, H, D = q.shape
+    if D != HEAD_DIM:
+        raise ValueError("head dim must be 128")
+    o = out if out is not None else torch.empty_like(q)
+    rc = _lib.kda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o), B, T, H,
+                                _dtype_code(q), float(scale), int(l2norm_qk), _stream(q.device))
+    _check(rc, "kda_recurrent_fwd")
     return o
 
 

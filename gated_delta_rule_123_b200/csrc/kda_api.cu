@@ -7,6 +7,9 @@
 
 namespace kda {
 
+int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
+                         cudaStream_t stream);
 int launch_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                        float* state, void* o, int B, int H, int dtype, float scale, int l2norm, cudaStream_t stream);
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -152,6 +155,23 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
         return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     const int rc = launch_decode_step(q, k, v, g, beta, state, o, B, H, dtype, scale, l2norm_qk,
                                       static_cast<cudaStream_t>(stream));
+    return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
+}
+
+int kda_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,
+                      void* o, int B, int T, int H, int dtype, float scale, int l2norm_qk, void* stream) {
+    t_last_error[0] = 0;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
+    if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if ((long long)B * H == 0 || T == 0) return KDA_OK;
+    if ((long long)B * H >= (1ll << 31) || (long long)B * T * H * kD >= (1ll << 40))
+        return fail(KDA_ERR_UNSUPPORTED, "too many heads or tokens");
+    if (!q || !k || !v || !g || !beta || !state || !o) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o))
+        return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (o == q || o == k || o == v) return fail(KDA_ERR_INVALID_ARG, "o must not alias q, k or v");
+    const int rc = launch_recurrent_fwd(q, k, v, g, beta, state, o, B, T, H, dtype, scale, l2norm_qk,
+                                        static_cast<cudaStream_t>(stream));
     return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
 }
 

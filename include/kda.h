@@ -198,6 +198,29 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *g,
                     void *stream);
 
 /* ------------------------------------------------------------------------
+ * kda_recurrent_fwd -- fused recurrent segments: T tokens per sequence, the
+ * state read once and written once.
+ *
+ * "Kimi Linear: An Expressive, Efficient Attention Architecture", section
+ * "Training and Inference": long prompts take the chunk kernel, single steps and
+ * segments of at most 64 tokens take a fused recurrent kernel, with a fixed
+ * recurrent state cached between calls.  This is that kernel: the residual
+ * form of kda_decode_step applied token by token, with each head's state held
+ * on chip across the segment.  Any T >= 0 is accepted; beyond about 64 tokens
+ * kda_chunk_fwd is faster.  T = 1 computes what kda_decode_step computes.
+ *
+ *   q, k, v   [B,T,H,128], dtype bf16 or fp32 (l2norm_qk as for kda_chunk_fwd).
+ *   g         fp32 [B,T,H,128] log decay;  beta fp32 [B,T,H].
+ *   state     fp32 [B,H,128,128], updated IN PLACE (the state after token T).
+ *   o         [B,T,H,128], same dtype as q; o_t = S_t^T (scale * q_t).  Must not
+ *             alias q, k or v.
+ * All arithmetic is fp32 on CUDA cores.  No workspace.
+ */
+int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      float *state, void *o, int B, int T, int H, int dtype, float scale, int l2norm_qk,
+                      void *stream);
+
+/* ------------------------------------------------------------------------
  * kda_layer_fwd -- the KDA layer around the operator (forward).
  *
  * "Kimi Linear: An Expressive, Efficient Attention Architecture", section
