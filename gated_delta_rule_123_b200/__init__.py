@@ -26,7 +26,7 @@ SYMBOLS = (
     "kda_status_string", "kda_head_dim", "kda_last_error", "kda_device_status",
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
-    "kda_gdn_chunk_fwd", "kda_recurrent_fwd",
+    "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
 )
 
 
@@ -65,8 +65,12 @@ def _load():
     lib.kda_recurrent_fwd.restype = i
     lib.kda_layer_fwd_workspace.argtypes = [i, i, i, i, i]
     lib.kda_layer_fwd_workspace.restype = sz
-    lib.kda_layer_fwd.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, i, i, vp, vp, vp, vp, sz, vp]
+    lib.kda_layer_fwd.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.kda_layer_fwd.restype = i
+    lib.kda_layer_decode_workspace.argtypes = [i, i, i, i, i]
+    lib.kda_layer_decode_workspace.restype = sz
+    lib.kda_layer_decode.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, vp, vp, i, i, vp, sz, vp]
+    lib.kda_layer_decode.restype = i
     lib.kda_set_trace_events.argtypes = [vp, i]
     lib.kda_set_trace_events.restype = i
     return lib
@@ -210,9 +214,18 @@ def layer_fwd_workspace_bytes(total_tokens, d_model, H, rank, num_seqs) -> int:
     return int(_lib.kda_layer_fwd_workspace(total_tokens, d_model, H, rank, num_seqs))
 
 
+def _layer_weights(packed: dict, d_model: int) -> LayerWeights:
+    return LayerWeights(packed["W_in"].data_ptr(), packed["W_aup"].data_ptr(), packed["W_gup"].data_ptr(),
+                        packed["conv_w"].data_ptr(), packed["norm_w"].data_ptr(), packed["W_o"].data_ptr(),
+                        d_model, packed["H"], packed["rank"])
+
+
 def layer_fwd(x, packed: dict, cu_seqlens, initial_state=None, output_final_state=True, out=None,
-              final_state=None, workspace=None):
-    """KDA layer forward (``kda_layer_fwd``).  x: [Ttot, d_model] bf16."""
+              final_state=None, workspace=None, conv_state_in=None, output_conv_state=False, conv_state_out=None):
+    """KDA layer forward (``kda_layer_fwd``).  x: [Ttot, d_model] bf16.
+
+    Returns (y, final_state or None, conv_state or None); the conv state is
+    [num_seqs, 3, 3*H*128] bf16 (the ShortConv cache)."""
     Ttot, d_model = x.shape
     H, rank = packed["H"], packed["rank"]
     nseq = cu_seqlens.numel() - 1
@@ -220,13 +233,34 @@ def layer_fwd(x, packed: dict, cu_seqlens, initial_state=None, output_final_stat
     fs = final_state
     if fs is None and output_final_state:
         fs = torch.empty((nseq, H, HEAD_DIM, HEAD_DIM), device=x.device, dtype=torch.float32)
-    lw = LayerWeights(packed["W_in"].data_ptr(), packed["W_aup"].data_ptr(), packed["W_gup"].data_ptr(),
-                      packed["conv_w"].data_ptr(), packed["norm_w"].data_ptr(), packed["W_o"].data_ptr(),
-                      d_model, H, rank)
+    cs = conv_state_out
+    if cs is None and output_conv_state:
+        cs = torch.empty((nseq, 3, 3 * H * HEAD_DIM), device=x.device, dtype=torch.bfloat16)
+    lw = _layer_weights(packed, d_model)
     wsz = layer_fwd_workspace_bytes(Ttot, d_model, H, rank, nseq)
     if workspace is None or workspace.numel() < wsz:
         workspace = torch.empty(max(wsz, 1), device=x.device, dtype=torch.uint8)
     rc = _lib.kda_layer_fwd(_ptr(x), ctypes.byref(lw), _ptr(cu_seqlens), nseq, Ttot, _ptr(initial_state), _ptr(fs),
-                            _ptr(y), _ptr(workspace), wsz, _stream(x.device))
+                            _ptr(conv_state_in), _ptr(cs), _ptr(y), _ptr(workspace), wsz, _stream(x.device))
     _check(rc, "kda_layer_fwd")
-    return y, fs
+    return y, fs, cs
+
+
+def layer_decode_workspace_bytes(B, T, d_model, H, rank) -> int:
+    return int(_lib.kda_layer_decode_workspace(B, T, d_model, H, rank))
+
+
+def layer_decode(x, packed: dict, conv_state, state, out=None, workspace=None):
+    """KDA layer on T new tokens per sequence (``kda_layer_decode``).  x: [B, T, d_model] bf16;
+    conv_state [B, 3, 3*H*128] bf16 and state [B, H, 128, 128] fp32 are updated in place."""
+    B, T, d_model = x.shape
+    H, rank = packed["H"], packed["rank"]
+    y = out if out is not None else torch.empty_like(x)
+    lw = _layer_weights(packed, d_model)
+    wsz = layer_decode_workspace_bytes(B, T, d_model, H, rank)
+    if workspace is None or workspace.numel() < wsz:
+        workspace = torch.empty(max(wsz, 1), device=x.device, dtype=torch.uint8)
+    rc = _lib.kda_layer_decode(_ptr(x), ctypes.byref(lw), _ptr(conv_state), _ptr(state), _ptr(y), B, T,
+                               _ptr(workspace), wsz, _stream(x.device))
+    _check(rc, "kda_layer_decode")
+    return y

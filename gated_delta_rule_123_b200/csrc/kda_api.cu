@@ -18,9 +18,12 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                      const char** why, int scalar_gate);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 size_t layer_workspace_bytes(int total_tokens, int d_model, int H, int rank, int num_seqs);
-int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int num_seqs, int total_tokens,
-                     const float* init, float* fin, void* y, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why);
+int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int nseq, int ntok,
+                     const float* init, float* fin, const void* conv_in, void* conv_out, void* y, void* ws,
+                     size_t ws_bytes, cudaStream_t stream, const char** why);
+size_t layer_decode_workspace_bytes(int B, int T, int d_model, int H, int rank);
+int launch_layer_decode(const void* x, const kda_layer_weights* w, void* conv_state, float* state, void* y, int B,
+                        int T, void* ws, size_t ws_bytes, cudaStream_t stream, const char** why);
 
 static thread_local char t_last_error[256] = "";
 thread_local cudaEvent_t* g_trace_events = nullptr;
@@ -180,26 +183,74 @@ size_t kda_layer_fwd_workspace(int total_tokens, int d_model, int H, int rank, i
     return layer_workspace_bytes(total_tokens, d_model, H, rank, num_seqs);
 }
 
-int kda_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu_seqlens, int num_seqs,
-                  int total_tokens, const float* initial_state, float* final_state, void* y, void* workspace,
-                  size_t workspace_bytes, void* stream) {
-    t_last_error[0] = 0;
+// Weight checks shared by the layer entry points.
+static int check_layer_weights(const kda_layer_weights* w) {
     if (!w) return fail(KDA_ERR_INVALID_ARG, "NULL weights");
-    if (w->d_model <= 0 || w->H <= 0 || w->rank <= 0 || total_tokens < 0 || num_seqs < 1)
-        return fail(KDA_ERR_INVALID_ARG, "bad sizes");
+    if (w->d_model <= 0 || w->H <= 0 || w->rank <= 0) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (w->d_model % 8 || w->rank % 8) return fail(KDA_ERR_UNSUPPORTED, "d_model and rank must be multiples of 8");
+    if (!w->W_in || !w->W_aup || !w->W_gup || !w->conv_w || !w->norm_w || !w->W_o)
+        return fail(KDA_ERR_INVALID_ARG, "NULL weight pointer");
+    if (!aligned16(w->W_in) || !aligned16(w->W_aup) || !aligned16(w->W_gup) || !aligned16(w->W_o))
+        return fail(KDA_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+    return KDA_OK;
+}
+
+int kda_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu_seqlens, int num_seqs,
+                  int total_tokens, const float* initial_state, float* final_state, const void* conv_state_in,
+                  void* conv_state_out, void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    const int wc = check_layer_weights(w);
+    if (wc != KDA_OK) return wc;
+    if (total_tokens < 0 || num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is required");
-    if (total_tokens == 0) return KDA_OK;
-    if (!x || !y || !w->W_in || !w->W_aup || !w->W_gup || !w->conv_w || !w->norm_w || !w->W_o)
-        return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
-    if (!aligned16(x) || !aligned16(y) || !aligned16(w->W_in) || !aligned16(w->W_aup) || !aligned16(w->W_gup) ||
-        !aligned16(w->W_o) || (initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)) ||
+        (conv_state_in && !aligned16(conv_state_in)) || (conv_state_out && !aligned16(conv_state_out)))
+        return fail(KDA_ERR_INVALID_ARG, "state pointers must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (total_tokens == 0) {  // every sequence is empty: the states pass through
+        const size_t sb = size_t(num_seqs) * w->H * kD * kD * sizeof(float);
+        const size_t cb = size_t(num_seqs) * 3 * 3 * w->H * kD * 2;
+        cudaError_t e = cudaSuccess;
+        if (final_state && final_state != initial_state)
+            e = initial_state ? cudaMemcpyAsync(final_state, initial_state, sb, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(final_state, 0, sb, s);
+        if (e == cudaSuccess && conv_state_out && conv_state_out != conv_state_in)
+            e = conv_state_in ? cudaMemcpyAsync(conv_state_out, conv_state_in, cb, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(conv_state_out, 0, cb, s);
+        return e == cudaSuccess ? KDA_OK : fail(KDA_ERR_CUDA, cudaGetErrorString(e));
+    }
+    if (!x || !y) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(y)) return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char* why = "";
+    const int rc = launch_layer_fwd(x, w, cu_seqlens, num_seqs, total_tokens, initial_state, final_state,
+                                    conv_state_in, conv_state_out, y, workspace, workspace_bytes, s, &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
+}
+
+size_t kda_layer_decode_workspace(int B, int T, int d_model, int H, int rank) {
+    if (B <= 0 || T <= 0 || d_model <= 0 || H <= 0 || rank <= 0) return 0;
+    return layer_decode_workspace_bytes(B, T, d_model, H, rank);
+}
+
+int kda_layer_decode(const void* x, const kda_layer_weights* w, void* conv_state, float* state, void* y, int B,
+                     int T, void* workspace, size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    const int wc = check_layer_weights(w);
+    if (wc != KDA_OK) return wc;
+    if (B < 0 || T < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if ((long long)B * T == 0) return KDA_OK;
+    if ((long long)B * T * (3 * w->H * kD + 2 * w->rank + w->H) >= (1ll << 31))
+        return fail(KDA_ERR_UNSUPPORTED, "too many tokens");
+    if (!x || !y || !conv_state || !state) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(y) || !aligned16(conv_state) || !aligned16(state))
         return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     const char* why = "";
-    const int rc = launch_layer_fwd(x, w, cu_seqlens, num_seqs, total_tokens, initial_state, final_state, y, workspace,
-                                    workspace_bytes, static_cast<cudaStream_t>(stream), &why);
+    const int rc = launch_layer_decode(x, w, conv_state, state, y, B, T, workspace, workspace_bytes,
+                                       static_cast<cudaStream_t>(stream), &why);
     return rc == KDA_OK ? KDA_OK : fail(rc, why);
 }
 

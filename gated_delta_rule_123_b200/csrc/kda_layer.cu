@@ -30,20 +30,30 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
                      const char** why, int scalar_gate);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
+int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
+                         cudaStream_t stream);
 
-__device__ __forceinline__ int seq_start_of(const int32_t* cu, int nseq, int t) {
-    int lo = 0, hi = nseq;  // find n with cu[n] <= t < cu[n+1]
+// Sequence of token t: packed (cu[n] <= t < cu[n+1]), or dense with seq_len
+// tokens per sequence when cu is NULL.
+__device__ __forceinline__ int seq_of(const int32_t* cu, int nseq, int seq_len, int t) {
+    if (!cu) return t / seq_len;
+    int lo = 0, hi = nseq;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (cu[mid] <= t) lo = mid; else hi = mid;
     }
-    return cu[lo];
+    return lo;
 }
+__device__ __forceinline__ int seq_begin(const int32_t* cu, int seq_len, int n) { return cu ? cu[n] : n * seq_len; }
 
-// One warp per (token, head, tensor in {q,k,v}); lane owns 4 channels.
+// One warp per (token, head, tensor in {q,k,v}); lane owns 4 channels.  Taps
+// before the sequence's first token in this call read the cached history
+// conv_in [nseq][3][3 H 128] (row 2 = the token just before), or zero.
 __global__ void conv_silu_norm_kernel(const __nv_bfloat16* __restrict__ z, int ldz,
                                       const __nv_bfloat16* __restrict__ conv_w, const int32_t* __restrict__ cu,
-                                      int nseq, int ntok, int H, __nv_bfloat16* __restrict__ q,
+                                      int nseq, int seq_len, int ntok, int H,
+                                      const __nv_bfloat16* __restrict__ conv_in, __nv_bfloat16* __restrict__ q,
                                       __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v) {
     const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -52,15 +62,18 @@ __global__ void conv_silu_norm_kernel(const __nv_bfloat16* __restrict__ z, int l
     const int which = int(wid % 3);
     const int h = int((wid / 3) % H);
     const int t = int(wid / (3LL * H));
-    const int s0 = seq_start_of(cu, nseq, t);
+    const int n = seq_of(cu, nseq, seq_len, t);
+    const int s0 = seq_begin(cu, seq_len, n);
     const int HD = H * kD;
     const int col0 = which * HD + h * kD + lane * 4;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int tt = t - 3 + j;
-        if (tt < s0) continue;
-        const uint2 raw = *reinterpret_cast<const uint2*>(z + (size_t)tt * ldz + col0);
+        if (tt < s0 && !conv_in) continue;
+        const __nv_bfloat16* src = tt >= s0 ? z + (size_t)tt * ldz + col0
+                                            : conv_in + ((size_t)n * 3 + (3 + tt - s0)) * (3 * HD) + col0;
+        const uint2 raw = *reinterpret_cast<const uint2*>(src);
         const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
         const float xv[4] = {__low2float(pr[0]), __high2float(pr[0]), __low2float(pr[1]), __high2float(pr[1])};
 #pragma unroll
@@ -82,6 +95,28 @@ __global__ void conv_silu_norm_kernel(const __nv_bfloat16* __restrict__ z, int l
     __nv_bfloat16* dst = which == 0 ? q : (which == 1 ? k : v);
     __nv_bfloat162 o2[2] = {__floats2bfloat162_rn(acc[0], acc[1]), __floats2bfloat162_rn(acc[2], acc[3])};
     *reinterpret_cast<uint2*>(dst + ((size_t)t * H + h) * kD + lane * 4) = *reinterpret_cast<uint2*>(o2);
+}
+
+// conv_out[n] = the last 3 conv inputs (q, k, v pre-activations) up to the end of
+// sequence n, oldest first, taken from this call's tokens and, for a sequence
+// shorter than 3, from the history conv_in (or zero).  One thread per (n,
+// column) reads its three sources before writing, so conv_out may equal conv_in.
+__global__ void conv_cache_out_kernel(const __nv_bfloat16* __restrict__ z, int ldz, const int32_t* __restrict__ cu,
+                                      int nseq, int seq_len, int C, const __nv_bfloat16* conv_in,
+                                      __nv_bfloat16* conv_out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)nseq * C) return;
+    const int n = int(i / C), c = int(i % C);
+    const int s0 = seq_begin(cu, seq_len, n), e0 = seq_begin(cu, seq_len, n + 1);
+    __nv_bfloat16 r[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int p = e0 - 3 + j;
+        r[j] = p >= s0 ? z[(size_t)p * ldz + c]
+                       : (conv_in ? conv_in[((size_t)n * 3 + (3 + p - s0)) * C + c] : __float2bfloat16_rn(0.f));
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) conv_out[((size_t)n * 3 + j) * C + c] = r[j];
 }
 
 // g = -softplus(a) (fp32, per channel); beta = sigmoid(b_raw) (per token, head).
@@ -188,7 +223,7 @@ constexpr size_t kLtWorkspace = 32u << 20;
 
 static size_t up256l(size_t x) { return (x + 255) & ~size_t(255); }
 
-static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nseq) {
+static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nseq, bool chunked = true) {
     (void)d_model;
     LayerPlan p{};
     p.HD = H * kD;
@@ -205,7 +240,7 @@ static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nse
     p.off_beta = off; off = up256l(off + size_t(ntok) * H * 4);
     p.off_o = off; off = up256l(off + tokHD * 2);
     p.off_lt = off; off = up256l(off + kLtWorkspace);
-    p.chunk_bytes = chunk_workspace_bytes(1, ntok, H, nseq, KDA_BF16, 0);
+    p.chunk_bytes = chunked ? chunk_workspace_bytes(1, ntok, H, nseq, KDA_BF16, 0) : 0;
     p.off_chunk = off; off = up256l(off + p.chunk_bytes);
     p.total = off;
     return p;
@@ -214,14 +249,22 @@ static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nse
 size_t layer_workspace_bytes(int ntok, int d_model, int H, int rank, int nseq) {
     return make_layer_plan(ntok, d_model, H, rank, nseq).total;
 }
+size_t layer_decode_workspace_bytes(int B, int T, int d_model, int H, int rank) {
+    return make_layer_plan(B * T, d_model, H, rank, B, false).total;
+}
 
-int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int nseq, int ntok,
-                     const float* init, float* fin, void* y, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why) {
+// Shared by the prefill (cu = packed offsets, KDA by the chunk kernels) and the
+// decode step (cu = NULL, B sequences of seq_len tokens, KDA by the fused
+// recurrent kernel on the state in place).
+static int layer_pipeline(const void* x, const kda_layer_weights* w, const int32_t* cu, int nseq, int seq_len,
+                          int ntok, const float* init, float* fin, float* state_inplace, const void* conv_in,
+                          void* conv_out, void* y, void* ws, size_t ws_bytes, cudaStream_t stream, const char** why) {
     const int H = w->H, D = w->d_model, R = w->rank;
-    const LayerPlan pl = make_layer_plan(ntok, D, H, R, nseq);
+    const bool decode = cu == nullptr;
+    const LayerPlan pl = make_layer_plan(ntok, D, H, R, nseq, !decode);
     if (!ws || ws_bytes < pl.total) {
-        *why = "workspace smaller than kda_layer_fwd_workspace()";
+        *why = decode ? "workspace smaller than kda_layer_decode_workspace()"
+                      : "workspace smaller than kda_layer_fwd_workspace()";
         return KDA_ERR_WORKSPACE;
     }
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -244,16 +287,32 @@ int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* c
     {
         const long long warps = (long long)ntok * H * 3;
         conv_silu_norm_kernel<<<unsigned((warps + 7) / 8), 256, 0, stream>>>(
-            zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu, nseq, ntok, H, q, k, v);
+            zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu, nseq, seq_len, ntok, H,
+            static_cast<const __nv_bfloat16*>(conv_in), q, k, v);
+    }
+    if (conv_out) {
+        const long long n = (long long)nseq * 3 * HD;
+        conv_cache_out_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(
+            zb, ldz, cu, nseq, seq_len, 3 * HD, static_cast<const __nv_bfloat16*>(conv_in),
+            static_cast<__nv_bfloat16*>(conv_out));
     }
     if (!gemm_bf16(zb + 3 * HD, ldz, w->W_aup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
         *why = "cuBLASLt alpha up-projection failed";
         return KDA_ERR_CUDA;
     }
     gates_kernel<<<1184, 256, 0, stream>>>(a, zb, ldz, 3 * HD + 2 * R, ntok, H, g, beta);
-    const int rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
-                                    b + pl.off_chunk, pl.chunk_bytes, stream, why, 0);
-    if (rc != KDA_OK) return rc;
+    if (decode) {
+        const int rc = launch_recurrent_fwd(q, k, v, g, beta, state_inplace, o, nseq, seq_len, H, KDA_BF16, 1.f, 0,
+                                            stream);
+        if (rc != KDA_OK) {
+            *why = "recurrent kernel launch failed";
+            return rc;
+        }
+    } else {
+        const int rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
+                                        b + pl.off_chunk, pl.chunk_bytes, stream, why, 0);
+        if (rc != KDA_OK) return rc;
+    }
     // output gate pre-activation reuses the alpha buffer
     if (!gemm_bf16(zb + 3 * HD + R, ldz, w->W_gup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
         *why = "cuBLASLt gate up-projection failed";
@@ -271,6 +330,19 @@ int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* c
         return KDA_ERR_CUDA;
     }
     return KDA_OK;
+}
+
+int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int nseq, int ntok,
+                     const float* init, float* fin, const void* conv_in, void* conv_out, void* y, void* ws,
+                     size_t ws_bytes, cudaStream_t stream, const char** why) {
+    return layer_pipeline(x, w, cu, nseq, 0, ntok, init, fin, nullptr, conv_in, conv_out, y, ws, ws_bytes, stream,
+                          why);
+}
+
+int launch_layer_decode(const void* x, const kda_layer_weights* w, void* conv_state, float* state, void* y, int B,
+                        int T, void* ws, size_t ws_bytes, cudaStream_t stream, const char** why) {
+    return layer_pipeline(x, w, nullptr, B, T, B * T, nullptr, nullptr, state, conv_state, conv_state, y, ws,
+                          ws_bytes, stream, why);
 }
 
 }  // namespace kda

@@ -229,8 +229,8 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
  * L2 norm of q and k; per-channel decay alpha = exp(-softplus(W_aup W_adown x))
  * (rank-128 low-rank projection); beta = sigmoid(W_b x); KDA (scale 1); per-head
  * RMSNorm (eps 1e-5, weight norm_w) times sigmoid(W_gup W_gdown x); output
- * projection.  Packed sequences: the convolution restarts from zero history at
- * every cu_seqlens start.
+ * projection.  Packed sequences: the convolution of each sequence starts from
+ * its cached history (conv_state_in) or, when that is NULL, from zero history.
  *
  * All weights are bf16 row-major "out x in" (y = x W^T) except conv_* and
  * norm_w:
@@ -243,6 +243,14 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
  *   x       bf16 [total_tokens, d_model];  y bf16 [total_tokens, d_model].
  *   cu_seqlens  device int32 [num_seqs+1] (required);
  *   initial_state / final_state as in kda_chunk_fwd (N = num_seqs).
+ *   conv_state_in / conv_state_out  bf16 [num_seqs, 3, 3*H*128] or NULL: the
+ *           ShortConv cache, i.e. the last three convolution inputs (the q, k, v
+ *           projections, in W_in's row order) before / at the end of each
+ *           sequence, oldest first.  A sequence shorter than three tokens keeps
+ *           the tail of its incoming history.  conv_state_out may equal
+ *           conv_state_in.  Together with final_state this is the fixed-size
+ *           cache the pages describe ("Training and Inference": KDA caches the
+ *           short-convolution state and the recurrent state).
  * Projections run on cuBLASLt (plain bf16 GEMMs, fp32 accumulate); everything
  * else runs in this library's kernels.
  */
@@ -261,8 +269,32 @@ typedef struct {
 size_t kda_layer_fwd_workspace(int total_tokens, int d_model, int H, int rank, int num_seqs);
 
 int kda_layer_fwd(const void *x, const kda_layer_weights *w, const int32_t *cu_seqlens, int num_seqs,
-                  int total_tokens, const float *initial_state, float *final_state, void *y,
+                  int total_tokens, const float *initial_state, float *final_state,
+                  const void *conv_state_in, void *conv_state_out, void *y,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * kda_layer_decode -- the layer on T new tokens per sequence from its cache.
+ *
+ * The inference path of "Kimi Linear" ("Training and Inference": single steps
+ * and segments of at most 64 tokens take the fused recurrent kernel; the KDA
+ * layer caches the short-convolution state and the recurrent state).  Same
+ * pipeline as kda_layer_fwd for B sequences of T tokens each, with the
+ * convolution reading its history from conv_state and the operator run by the
+ * fused recurrent kernel (kda_recurrent_fwd) on state; both caches are updated
+ * in place, so repeated calls continue the sequences.  After a kda_layer_fwd
+ * prefill, its final_state and conv_state_out are the caches to pass here.
+ *
+ *   x           bf16 [B, T, d_model];   y bf16 [B, T, d_model].
+ *   conv_state  bf16 [B, 3, 3*H*128], in place (layout as in kda_layer_fwd).
+ *   state       fp32 [B, H, 128, 128], in place.
+ *   workspace   at least kda_layer_decode_workspace(B, T, d_model, H, rank)
+ *               bytes, 256-byte aligned.
+ */
+size_t kda_layer_decode_workspace(int B, int T, int d_model, int H, int rank);
+
+int kda_layer_decode(const void *x, const kda_layer_weights *w, void *conv_state, float *state, void *y,
+                     int B, int T, void *workspace, size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

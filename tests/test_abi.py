@@ -80,7 +80,43 @@ def test_decode_validation_rejects_before_launch(kda):
 def test_layer_validation_rejects_before_launch(kda):
     lib = kda.lib()
     w = kda.LayerWeights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 2048, 16, 128)
-    assert lib.kda_layer_fwd(1 << 20, None, 1 << 21, 8, 64, None, None, 1 << 22, None, 0, None) == kda.KDA_ERR_INVALID_ARG
-    assert lib.kda_layer_fwd(1 << 20, ctypes.byref(w), None, 8, 64, None, None, 1 << 22, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    p, y = 1 << 20, 1 << 22
+    assert lib.kda_layer_fwd(p, None, 1 << 21, 8, 64, None, None, None, None, y, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_layer_fwd(p, ctypes.byref(w), None, 8, 64, None, None, None, None, y, None, 0, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    # misaligned conv cache
+    assert lib.kda_layer_fwd(p, ctypes.byref(w), 1 << 21, 8, 64, None, None, p + 2, None, y, None, 0, None) == \
+        kda.KDA_ERR_INVALID_ARG
     w.d_model = 2047
-    assert lib.kda_layer_fwd(1 << 20, ctypes.byref(w), 1 << 21, 8, 64, None, None, 1 << 22, None, 0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_layer_fwd(p, ctypes.byref(w), 1 << 21, 8, 64, None, None, None, None, y, None, 0, None) == \
+        kda.KDA_ERR_UNSUPPORTED
+
+
+def test_layer_decode_validation_rejects_before_launch(kda):
+    lib = kda.lib()
+    w = kda.LayerWeights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 2048, 16, 128)
+    p = 1 << 20
+    assert lib.kda_layer_decode(p, None, p, p, p, 4, 1, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_layer_decode(p, ctypes.byref(w), None, p, p, 4, 1, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_layer_decode(p, ctypes.byref(w), p, p + 4, p, 4, 1, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_layer_decode(p, ctypes.byref(w), p, p, p, -1, 1, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_layer_decode(p, ctypes.byref(w), p, p, p, 0, 1, None, 0, None) == kda.KDA_OK  # nothing to do
+    assert kda.layer_decode_workspace_bytes(4, 1, 2048, 16, 128) > 0
+
+
+def test_recurrent_validation_rejects_before_launch(kda):
+    lib = kda.lib()
+    p = 1 << 20
+    assert lib.kda_recurrent_fwd(p, p, p, p, p, None, p + 256, 2, 3, 2, 0, 1.0, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_recurrent_fwd(p, p, p, p, p, p, p, 2, 3, 2, 0, 1.0, 0, None) == kda.KDA_ERR_INVALID_ARG  # o aliases q
+    assert lib.kda_recurrent_fwd(p, p, p, p, p, p, p + 256, 2, 3, 2, 7, 1.0, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_recurrent_fwd(p, p, p, p, p, p, p + 256, 2, 0, 2, 0, 1.0, 0, None) == kda.KDA_OK  # T = 0
+
+
+def test_gdn_validation_rejects_before_launch(kda):
+    lib = kda.lib()
+    p = 1 << 20
+    assert lib.kda_gdn_chunk_fwd(p, p, p, p, p, None, None, p + 256, None, 3, 1, 64, 2, 0, 1.0, 0, None, 0,
+                                 None) == kda.KDA_ERR_INVALID_ARG  # num_seqs without cu_seqlens
+    assert lib.kda_gdn_chunk_fwd(p, p, p, p, p, None, None, p, None, 0, 1, 64, 2, 0, 1.0, 0, None, 0,
+                                 None) == kda.KDA_ERR_INVALID_ARG  # o aliases q

@@ -29,7 +29,7 @@ def run_layer(kda, d_model, H, Ttot, nseq, rank, seed, s0=True, check_seqs=None)
     Wd = {n: t.to(dev) for n, t in W.items()}
     packed = kda.pack_layer_weights(Wd)
     cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
-    y, fs = kda.layer_fwd(x.to(dev), packed, cu_d, initial_state=None if S0 is None else S0.to(dev))
+    y, fs, _ = kda.layer_fwd(x.to(dev), packed, cu_d, initial_state=None if S0 is None else S0.to(dev))
     torch.cuda.synchronize()
     assert kda.device_status() == 0
     Wn = {n: f64(t) for n, t in W.items()}
