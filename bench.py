@@ -319,6 +319,33 @@ def run_ours(args):
     assert kda.device_status() == 0
     gdn_bytes = GDN_BYTES_PER_TOKEN_HEAD * T * H_PREFILL
 
+    # untied DPLR comparison kernel: at the pages' comparison shape (B=1, H=16, T; one CTA per head,
+    # no segment scan) and, against KDA, at a shape where neither kernel segments (B=16, H=16, T=4096)
+    def time_calls(fn, n):
+        for _ in range(2):
+            fn()
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(n):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(start.elapsed_time(end) / n)
+
+    dp = synth.dplr_inputs(B=1, H=H_PREFILL, T=T, s0_std=0.02, seed=cfg["seed"] + 11, device=dev)
+    dargs = [dp[n] for n in ("q", "k", "v", "a", "b", "g", "beta")]
+    dplr_ms = time_calls(lambda: kda.dplr_chunk_fwd(*dargs, initial_state=dp["s0"], out=o, final_state=fs), 3)
+    del dp, dargs
+    eq = synth.dplr_inputs(B=16, H=H_PREFILL, T=4096, s0_std=0.02, seed=cfg["seed"] + 12, device=dev)
+    eo_, efs = torch.empty_like(eq["q"]), torch.empty_like(eq["s0"])
+    eq_dplr_ms = time_calls(lambda: kda.dplr_chunk_fwd(*(eq[n] for n in ("q", "k", "v", "a", "b", "g", "beta")),
+                                                       initial_state=eq["s0"], out=eo_, final_state=efs), 5)
+    eq_kda_ms = time_calls(lambda: kda.chunk_fwd(*(eq[n] for n in ("q", "k", "v", "g", "beta")),
+                                                 initial_state=eq["s0"], out=eo_, final_state=efs), 5)
+    del eq, eo_, efs
+    assert kda.device_status() == 0
+
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -372,6 +399,11 @@ def run_ours(args):
             "recurrent": {"workload": f"B={B} H={H} segments of {rT} tokens, fp32 state in place",
                           "us_per_call": rec_us, "tokens_per_s": world * B * rT / (rec_us / 1e6),
                           "us_per_token": rec_us / rT},
+            "dplr": {"workload": f"untied DPLR prefill B=1 H=16 T={T} (one CTA per head, no segment scan)",
+                     "ms_per_step": dplr_ms, "tokens_per_s": world * T / (dplr_ms / 1e3),
+                     "equal_parallelism": {"workload": "B=16 H=16 T=4096, neither kernel segments",
+                                           "dplr_ms": eq_dplr_ms, "kda_ms": eq_kda_ms,
+                                           "dplr_over_kda": eq_dplr_ms / eq_kda_ms}},
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,

@@ -27,6 +27,7 @@ SYMBOLS = (
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
+    "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd",
 )
 
 
@@ -63,6 +64,10 @@ def _load():
     lib.kda_decode_step.restype = i
     lib.kda_recurrent_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.kda_recurrent_fwd.restype = i
+    lib.kda_dplr_chunk_fwd_workspace.argtypes = [i, i, i, i, i]
+    lib.kda_dplr_chunk_fwd_workspace.restype = sz
+    lib.kda_dplr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    lib.kda_dplr_chunk_fwd.restype = i
     lib.kda_layer_fwd_workspace.argtypes = [i, i, i, i, i]
     lib.kda_layer_fwd_workspace.restype = sz
     lib.kda_layer_fwd.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -185,6 +190,32 @@ def decode_step(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None):
                               _dtype_code(q), float(scale), int(l2norm_qk), _stream(q.device))
     _check(rc, "kda_decode_step")
     return o
+
+
+def dplr_chunk_fwd(q, k, v, a, b, g, beta, initial_state=None, cu_seqlens=None, scale=1.0,
+                   output_final_state=True, out=None, final_state=None, workspace=None):
+    """Untied DPLR chunked prefill (``kda_dplr_chunk_fwd``): S = (I - a b^T) Diag(e^g) S + beta k v^T.
+
+    q, k, v, a, b, g: [B,T,H,128] (or [1,Ttot,H,128] with cu_seqlens); beta: [B,T,H].
+    Returns (o, final_state or None)."""
+    B, T, H, D = q.shape
+    if D != HEAD_DIM:
+        raise ValueError("head dim must be 128")
+    dt = _dtype_code(q)
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else nseq
+    o = out if out is not None else torch.empty_like(q)
+    fs = final_state
+    if fs is None and output_final_state:
+        fs = torch.empty((N, H, D, D), device=q.device, dtype=torch.float32)
+    wsz = int(_lib.kda_dplr_chunk_fwd_workspace(B, T, H, nseq, dt))
+    if workspace is None or workspace.numel() < wsz:
+        workspace = torch.empty(max(wsz, 1), device=q.device, dtype=torch.uint8)
+    rc = _lib.kda_dplr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(g), _ptr(beta),
+                                 _ptr(initial_state), _ptr(fs), _ptr(o), _ptr(cu_seqlens), nseq, B, T, H, dt,
+                                 float(scale), _ptr(workspace), wsz, _stream(q.device))
+    _check(rc, "kda_dplr_chunk_fwd")
+    return o, fs
 
 
 def recurrent_fwd(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None):

@@ -7,6 +7,11 @@
 
 namespace kda {
 
+size_t dplr_workspace_bytes(int B, int T, int H, int num_seqs, int dtype);
+int launch_dplr_chunk_fwd(const void* q, const void* k, const void* v, const void* a, const void* b, const float* g,
+                          const float* beta, const float* init, float* fin, void* o, const int32_t* cu, int num_seqs,
+                          int B, int T, int H, int dtype, float scale, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          const char** why);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
                          cudaStream_t stream);
@@ -159,6 +164,54 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
     const int rc = launch_decode_step(q, k, v, g, beta, state, o, B, H, dtype, scale, l2norm_qk,
                                       static_cast<cudaStream_t>(stream));
     return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
+}
+
+size_t kda_dplr_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;
+    return dplr_workspace_bytes(B, T, H, num_seqs, dtype);
+}
+
+int kda_dplr_chunk_fwd(const void* q, const void* k, const void* v, const void* a, const void* b, const float* g,
+                       const float* beta, const float* initial_state, float* final_state, void* o,
+                       const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dtype, float scale,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
+    if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if (cu_seqlens) {
+        if (B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1");
+        if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires num_seqs >= 1");
+    } else if (num_seqs != 0) {
+        return fail(KDA_ERR_INVALID_ARG, "num_seqs must be 0 for dense input");
+    }
+    const long long N = cu_seqlens ? num_seqs : B;
+    if ((long long)(cu_seqlens ? 1 : B) * T * H * kD >= (1ll << 31))
+        return fail(KDA_ERR_UNSUPPORTED, "more than 2^31 elements per token tensor");
+    if (N > 65535 || H > 65535) return fail(KDA_ERR_UNSUPPORTED, "more than 65535 sequences or heads");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((long long)T * H == 0 || N == 0) {
+        if (final_state && N * H > 0) {
+            const size_t bytes = size_t(N) * H * kD * kD * sizeof(float);
+            cudaError_t e = initial_state ? (initial_state == final_state
+                                                 ? cudaSuccess
+                                                 : cudaMemcpyAsync(final_state, initial_state, bytes,
+                                                                   cudaMemcpyDeviceToDevice, s))
+                                          : cudaMemsetAsync(final_state, 0, bytes, s);
+            if (e != cudaSuccess) return fail(KDA_ERR_CUDA, cudaGetErrorString(e));
+        }
+        return KDA_OK;
+    }
+    if (!q || !k || !v || !a || !b || !g || !beta || !o) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned16(b) || !aligned16(g) ||
+        !aligned16(o) || (initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (o == q || o == k || o == v || o == a || o == b) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char* why = "";
+    const int rc = launch_dplr_chunk_fwd(q, k, v, a, b, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs,
+                                         B, T, H, dtype, scale, workspace, workspace_bytes, s, &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
 }
 
 int kda_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,

@@ -2,6 +2,7 @@
 // word shared by every kernel).
 #include "kda_api.cu"
 #include "kda_chunk.cu"
+#include "kda_dplr.cu"
 #include "kda_decode.cu"
 #include "kda_layer.cu"
 #include "kda_noalloc.cu"

@@ -154,6 +154,38 @@ int kda_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *
                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * kda_dplr_chunk_fwd -- chunkwise prefill of the general (untied) DPLR
+ * recurrence, the comparison point for KDA.
+ *
+ *     S_t = (I - a_t b_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T (scale * q_t),
+ * with a_t, b_t free vectors per (token, head).  "Kimi Linear: An Expressive,
+ * Efficient Attention Architecture", section "Chunkwise Algorithm": KDA is the
+ * constrained DPLR transition whose low-rank pair is tied to the key (a = beta k,
+ * b = k here), which halves the gated gram matrices per chunk (four become two)
+ * and is what the pages' 64K kernel timing compares against.  This entry point
+ * computes the untied form with the same chunk size, tiling and numerics as
+ * kda_chunk_fwd, so the two can be timed against each other.
+ *
+ *   q, k, v, a, b  [B,T,H,128] (or [1,Ttot,H,128] with cu_seqlens), bf16 or fp32.
+ *   g              fp32, same shape: log decay (<= 0; below -1e4 treated as -1e4).
+ *   beta           fp32 [B,T,H].
+ *   initial_state, final_state, o, cu_seqlens, num_seqs, scale: as in
+ *   kda_chunk_fwd (no in-kernel L2 norm: normalise a, b, k, q beforehand).
+ *   workspace      at least kda_dplr_chunk_fwd_workspace(B, T, H, num_seqs, dtype)
+ *                  bytes, 256-byte aligned.
+ * Each (sequence, head) runs in one CTA, chunk after chunk: unlike
+ * kda_chunk_fwd there is no segment scan, so few long sequences use few SMs.
+ * Up to 65535 sequences and 65535 heads.
+ */
+size_t kda_dplr_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype);
+
+int kda_dplr_chunk_fwd(const void *q, const void *k, const void *v, const void *a, const void *b, const float *g,
+                       const float *beta, const float *initial_state, float *final_state, void *o,
+                       const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dtype, float scale,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
  * No counterpart on the pages: this is a library convenience.  Some callers

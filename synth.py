@@ -75,6 +75,22 @@ def op_inputs(B, H, T, dtype=torch.bfloat16, gate_scale=0.1, s0_std=None, seed=0
     return out
 
 
+def dplr_inputs(B, H, T, dtype=torch.bfloat16, gate_scale=0.1, s0_std=None, seed=0, device="cpu",
+                cu_seqlens=None, **_):
+    """Inputs of the untied DPLR recurrence S = (I - a b^T) Diag(e^g) S + beta k v^T:
+    the KDA inputs of ``op_inputs`` (same seed, same draws) plus a = sqrt(beta) k and
+    b = sqrt(beta) bh, with bh an independent unit vector per (token, head), drawn
+    after everything else.  bh = k would give back KDA."""
+    out = op_inputs(B, H, T, dtype=dtype, gate_scale=gate_scale, s0_std=s0_std, seed=seed, device=device,
+                    cu_seqlens=cu_seqlens)
+    gen = _gen(seed * 7919 + 17, device)
+    bh = _unit_heads(torch.randn(out["q"].shape, generator=gen, device=device))
+    sb = out["beta"].sqrt()[..., None]
+    out["a"] = (sb * out["k"].float()).to(dtype)
+    out["b"] = (sb * bh).to(dtype)
+    return out
+
+
 def random_cu_seqlens(Ttot: int, nseq: int, seed: int) -> list:
     """nseq packed sequences: nseq-1 distinct uniform cut points in [1, Ttot-1]."""
     gen = _gen(seed, "cpu")
