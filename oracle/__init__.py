@@ -26,6 +26,8 @@ Parts:
 * ``dplr_recurrent``          untied generic DPLR recurrence, product form (C).
 * ``kda_chunkwise``           naive chunkwise evaluation (numpy), any chunk size.
 * ``kda_layer``               the full KDA layer (numpy + the recurrence).
+* ``kda_recurrent_backward``  reverse mode of the recurrence (numpy): dq, dk, dv,
+                              dg, dbeta and the initial-state gradient.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against facts the
 pages and plain mathematics fix (special cases, closed forms, invariants, an
@@ -39,6 +41,7 @@ import subprocess
 
 import numpy as np
 
+from .backward import kda_recurrent_backward  # noqa: F401
 from .chunkwise import kda_chunkwise  # noqa: F401
 from .layer import kda_layer, layer_reference_parts  # noqa: F401
 
