@@ -346,6 +346,16 @@ def run_ours(args):
     del eq, eo_, efs
     assert kda.device_status() == 0
 
+    # backward (recurrent reverse mode) on B=1 H=16 T=8192, all six gradients
+    bT = 8192
+    bw = synth.op_inputs(B=1, H=H_PREFILL, T=bT, s0_std=0.02, seed=cfg["seed"] + 13, device=dev)
+    bdo = torch.randn(bw["q"].shape, device=dev, generator=torch.Generator(device=dev).manual_seed(7)).to(bw["q"].dtype)
+    bws = torch.empty(kda.lib().kda_recurrent_bwd_workspace(1, bT, H_PREFILL), device=dev, dtype=torch.uint8)
+    bwd_ms = time_calls(lambda: kda.recurrent_bwd(bw["q"], bw["k"], bw["v"], bw["g"], bw["beta"], bdo,
+                                                  initial_state=bw["s0"], workspace=bws), 2)
+    del bw, bdo, bws
+    assert kda.device_status() == 0
+
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -404,6 +414,8 @@ def run_ours(args):
                      "equal_parallelism": {"workload": "B=16 H=16 T=4096, neither kernel segments",
                                            "dplr_ms": eq_dplr_ms, "kda_ms": eq_kda_ms,
                                            "dplr_over_kda": eq_dplr_ms / eq_kda_ms}},
+            "backward": {"workload": "B=1 H=16 T=8192: dq, dk, dv, dg, dbeta, dS0 by recurrent reverse mode",
+                         "ms_per_call": bwd_ms, "tokens_per_s": world * bT / (bwd_ms / 1e3)},
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,

@@ -27,7 +27,7 @@ SYMBOLS = (
     "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
-    "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd",
+    "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
 )
 
 
@@ -68,6 +68,10 @@ def _load():
     lib.kda_dplr_chunk_fwd_workspace.restype = sz
     lib.kda_dplr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     lib.kda_dplr_chunk_fwd.restype = i
+    lib.kda_recurrent_bwd_workspace.argtypes = [i, i, i]
+    lib.kda_recurrent_bwd_workspace.restype = sz
+    lib.kda_recurrent_bwd.argtypes = [vp] * 14 + [i, i, i, i, f, vp, sz, vp]
+    lib.kda_recurrent_bwd.restype = i
     lib.kda_layer_fwd_workspace.argtypes = [i, i, i, i, i]
     lib.kda_layer_fwd_workspace.restype = sz
     lib.kda_layer_fwd.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -216,6 +220,26 @@ def dplr_chunk_fwd(q, k, v, a, b, g, beta, initial_state=None, cu_seqlens=None, 
                                  float(scale), _ptr(workspace), wsz, _stream(q.device))
     _check(rc, "kda_dplr_chunk_fwd")
     return o, fs
+
+
+def recurrent_bwd(q, k, v, g, beta, d_o, initial_state=None, d_final_state=None, scale=1.0, workspace=None):
+    """Gradients of the recurrence (``kda_recurrent_bwd``).  Returns (dq, dk, dv, dg, dbeta, d_initial_state),
+    all fp32; q, k, v, d_o [B,T,H,128] (bf16 or fp32), g [B,T,H,128], beta [B,T,H]."""
+    B, T, H, D = q.shape
+    if D != HEAD_DIM:
+        raise ValueError("head dim must be 128")
+    dev = q.device
+    dq, dk, dv, dg = (torch.empty((B, T, H, D), device=dev, dtype=torch.float32) for _ in range(4))
+    db = torch.empty((B, T, H), device=dev, dtype=torch.float32)
+    ds0 = torch.empty((B, H, D, D), device=dev, dtype=torch.float32)
+    wsz = int(_lib.kda_recurrent_bwd_workspace(B, T, H))
+    if workspace is None or workspace.numel() < wsz:
+        workspace = torch.empty(max(wsz, 1), device=dev, dtype=torch.uint8)
+    rc = _lib.kda_recurrent_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(d_o),
+                                _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(ds0),
+                                B, T, H, _dtype_code(q), float(scale), _ptr(workspace), wsz, _stream(dev))
+    _check(rc, "kda_recurrent_bwd")
+    return dq, dk, dv, dg, db, ds0
 
 
 def recurrent_fwd(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None):

@@ -12,6 +12,11 @@ int launch_dplr_chunk_fwd(const void* q, const void* k, const void* v, const voi
                           const float* beta, const float* init, float* fin, void* o, const int32_t* cu, int num_seqs,
                           int B, int T, int H, int dtype, float scale, void* ws, size_t ws_bytes, cudaStream_t stream,
                           const char** why);
+size_t recurrent_bwd_workspace_bytes(int B, int T, int H);
+int launch_recurrent_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         const float* init, const void* dout, const float* dfinal, float* dq, float* dk, float* dv,
+                         float* dg, float* dbeta, float* dinit, int B, int Tn, int H, int dtype, float scale,
+                         void* ws, size_t ws_bytes, cudaStream_t stream, const char** why);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
                          cudaStream_t stream);
@@ -164,6 +169,45 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
     const int rc = launch_decode_step(q, k, v, g, beta, state, o, B, H, dtype, scale, l2norm_qk,
                                       static_cast<cudaStream_t>(stream));
     return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
+}
+
+size_t kda_recurrent_bwd_workspace(int B, int T, int H) {
+    if (B < 0 || T < 0 || H < 0) return 0;
+    return recurrent_bwd_workspace_bytes(B, T, H);
+}
+
+int kda_recurrent_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* initial_state, const void* d_o, const float* d_final_state, float* dq, float* dk,
+                      float* dv, float* dg, float* dbeta, float* d_initial_state, int B, int T, int H, int dtype,
+                      float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    t_last_error[0] = 0;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return fail(KDA_ERR_INVALID_ARG, "dtype must be KDA_BF16 or KDA_FP32");
+    if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((long long)B * H == 0) return KDA_OK;
+    if ((long long)B * H >= (1ll << 31) || (long long)B * T * H * kD >= (1ll << 40))
+        return fail(KDA_ERR_UNSUPPORTED, "too many heads or tokens");
+    if (T == 0) {  // the initial-state gradient is the final-state gradient
+        if (d_initial_state) {
+            const size_t bytes = size_t(B) * H * kD * kD * sizeof(float);
+            const cudaError_t e = d_final_state ? cudaMemcpyAsync(d_initial_state, d_final_state, bytes,
+                                                                  cudaMemcpyDeviceToDevice, s)
+                                                : cudaMemsetAsync(d_initial_state, 0, bytes, s);
+            if (e != cudaSuccess) return fail(KDA_ERR_CUDA, cudaGetErrorString(e));
+        }
+        return KDA_OK;
+    }
+    if (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta)
+        return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    const void* p16[] = {q, k, v, g, d_o, dq, dk, dv, dg, initial_state, d_final_state, d_initial_state};
+    for (const void* ptr : p16)
+        if (ptr && !aligned16(ptr)) return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char* why = "";
+    const int rc = launch_recurrent_bwd(q, k, v, g, beta, initial_state, d_o, d_final_state, dq, dk, dv, dg, dbeta,
+                                        d_initial_state, B, T, H, dtype, scale, workspace, workspace_bytes, s, &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
 }
 
 size_t kda_dplr_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype) {

@@ -4,5 +4,6 @@
 #include "kda_chunk.cu"
 #include "kda_dplr.cu"
 #include "kda_decode.cu"
+#include "kda_backward.cu"
 #include "kda_layer.cu"
 #include "kda_noalloc.cu"

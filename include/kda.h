@@ -253,6 +253,36 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
                       void *stream);
 
 /* ------------------------------------------------------------------------
+ * kda_recurrent_bwd -- gradients of the operator (reverse mode).
+ *
+ * For a loss L with dL/do = d_o and dL/dS_T = d_final_state, computes dL/dq,
+ * dL/dk, dL/dv, dL/dg, dL/dbeta and dL/dS_0 of the recurrence above.  Training
+ * needs them ("Kimi Linear: An Expressive, Efficient Attention Architecture",
+ * section "Training and Inference"; the pages' public-code audit lists
+ * q/k/v/g/beta and initial-state gradient tests).  The reverse of each
+ * recurrent step is evaluated exactly in fp32 on CUDA cores: one CTA per
+ * (sequence, head) runs the forward once storing the state every 64 tokens,
+ * then walks the chunks backwards, recomputing each chunk's states.  It is the
+ * reference-speed backward (about 2x the token-serial forward work per token);
+ * a chunked tensor-core backward is not part of this build.
+ *
+ *   q, k, v, d_o   [B,T,H,128], dtype bf16 or fp32 (q, k not normalised here).
+ *   g              fp32 [B,T,H,128];  beta fp32 [B,T,H].
+ *   initial_state  fp32 [B,H,128,128] or NULL (zero);  d_final_state likewise.
+ *   dq, dk, dv, dg fp32 [B,T,H,128];  dbeta fp32 [B,T,H];
+ *   d_initial_state fp32 [B,H,128,128] or NULL (not written).
+ *   workspace      at least kda_recurrent_bwd_workspace(B, T, H) bytes
+ *                  ((ceil(T/64) + 64) x 64 KiB per (sequence, head)), 256-byte aligned.
+ * Dense batches only (no cu_seqlens).
+ */
+size_t kda_recurrent_bwd_workspace(int B, int T, int H);
+
+int kda_recurrent_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      const float *initial_state, const void *d_o, const float *d_final_state, float *dq,
+                      float *dk, float *dv, float *dg, float *dbeta, float *d_initial_state, int B, int T, int H,
+                      int dtype, float scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * kda_layer_fwd -- the KDA layer around the operator (forward).
  *
  * "Kimi Linear: An Expressive, Efficient Attention Architecture", section
