@@ -356,6 +356,23 @@ def run_ours(args):
     del bw, bdo, bws
     assert kda.device_status() == 0
 
+    # the KDA layer: d_model=2048, H=16, rank 128, 65536 packed tokens in 8 sequences, random-init weights
+    lc = synth.LAYER_65K
+    lx, lW, lcu = synth.layer_inputs(d_model=lc["d_model"], H=lc["H"], Ttot=lc["Ttot"], nseq=lc["nseq"],
+                                     rank=lc["rank"], seed=lc["seed"] + rank, device=dev)
+    lpk = kda.pack_layer_weights(lW)
+    lcu_d = torch.tensor(lcu, dtype=torch.int32, device=dev)
+    ly = torch.empty_like(lx)
+    lfs = torch.empty((lc["nseq"], lc["H"], D, D), device=dev, dtype=torch.float32)
+    lws = torch.empty(kda.layer_fwd_workspace_bytes(lc["Ttot"], lc["d_model"], lc["H"], lc["rank"], lc["nseq"]),
+                      device=dev, dtype=torch.uint8)
+    layer_ms = time_calls(lambda: kda.layer_fwd(lx, lpk, lcu_d, out=ly, final_state=lfs, workspace=lws), 5)
+    HDl, dm, rk = lc["H"] * D, lc["d_model"], lc["rank"]
+    gemm_flop = 2 * lc["Ttot"] * (dm * (3 * HDl + 2 * rk + lc["H"]) + 2 * rk * HDl + HDl * dm)
+    layer_flop = gemm_flop + FLOP_PER_TOKEN_HEAD * lc["Ttot"] * lc["H"]
+    del lx, lW, lpk, ly, lfs, lws
+    assert kda.device_status() == 0
+
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -416,6 +433,11 @@ def run_ours(args):
                                            "dplr_over_kda": eq_dplr_ms / eq_kda_ms}},
             "backward": {"workload": "B=1 H=16 T=8192: dq, dk, dv, dg, dbeta, dS0 by recurrent reverse mode",
                          "ms_per_call": bwd_ms, "tokens_per_s": world * bT / (bwd_ms / 1e3)},
+            "layer": {"workload": "KDA layer d_model=2048 H=16 rank=128, 65536 packed tokens (8 sequences), "
+                                  "random-init bf16 weights", "ms_per_call": layer_ms,
+                      "tokens_per_s": world * lc["Ttot"] / (layer_ms / 1e3),
+                      "tflops": layer_flop / (layer_ms / 1e3) / 1e12, "gemm_tflop_per_call": gemm_flop / 1e12,
+                      "tensor_peak_tflops": tc_peak, "frac": layer_flop / (layer_ms / 1e3) / 1e12 / tc_peak},
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,
