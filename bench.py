@@ -154,6 +154,29 @@ def run_reference(args):
     return 0
 
 
+def time_layer(kda, synth, dev, rank, time_calls, tc_peak, world):
+    """The KDA layer: d_model=2048, H=16, rank 128, 65536 packed tokens in 8 sequences, random-init weights."""
+    import torch
+    lc = synth.LAYER_65K
+    lx, lW, lcu = synth.layer_inputs(d_model=lc["d_model"], H=lc["H"], Ttot=lc["Ttot"], nseq=lc["nseq"],
+                                     rank=lc["rank"], seed=lc["seed"] + rank, device=dev)
+    lpk = kda.pack_layer_weights(lW)
+    lcu_d = torch.tensor(lcu, dtype=torch.int32, device=dev)
+    ly = torch.empty_like(lx)
+    lfs = torch.empty((lc["nseq"], lc["H"], D, D), device=dev, dtype=torch.float32)
+    lws = torch.empty(kda.layer_fwd_workspace_bytes(lc["Ttot"], lc["d_model"], lc["H"], lc["rank"], lc["nseq"]),
+                      device=dev, dtype=torch.uint8)
+    ms = time_calls(lambda: kda.layer_fwd(lx, lpk, lcu_d, out=ly, final_state=lfs, workspace=lws), 5)
+    HDl, dm, rk = lc["H"] * D, lc["d_model"], lc["rank"]
+    gemm_flop = 2 * lc["Ttot"] * (dm * (3 * HDl + 2 * rk + lc["H"]) + 2 * rk * HDl + HDl * dm)
+    flop = gemm_flop + FLOP_PER_TOKEN_HEAD * lc["Ttot"] * lc["H"]
+    return {"workload": "KDA layer d_model=2048 H=16 rank=128, 65536 packed tokens (8 sequences), "
+                        "random-init bf16 weights", "ms_per_call": ms,
+            "tokens_per_s": world * lc["Ttot"] / (ms / 1e3), "tflops": flop / (ms / 1e3) / 1e12,
+            "gemm_tflop_per_call": gemm_flop / 1e12, "tensor_peak_tflops": tc_peak,
+            "frac": flop / (ms / 1e3) / 1e12 / tc_peak}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -196,6 +219,29 @@ def run_ours(args):
     def step():
         kda.chunk_fwd(q, k, v, g, beta, initial_state=s0, out=o, final_state=fs, workspace=ws)
 
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def time_calls(fn, n):
+        for _ in range(2):
+            fn()
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(n):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(start.elapsed_time(end) / n)
+
+    if args.layer_only:
+        layer = time_layer(kda, synth, dev, rank, time_calls, tc_peak, world)
+        if rank == 0:
+            print(json.dumps({"metric": "KDA layer tokens/s", "value": layer["tokens_per_s"], "unit": "tokens/s",
+                              "config": {"workload": layer["workload"]}, "layer": layer}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
     sampler = ClockSampler(local)
     sampler.start()
     t_w = time.perf_counter()
@@ -210,7 +256,6 @@ def run_ours(args):
 
     # timed region: K steps, per-kernel trace events on the launching stream
     traces = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     start.record(stream)
@@ -321,17 +366,6 @@ def run_ours(args):
 
     # untied DPLR comparison kernel: at the pages' comparison shape (B=1, H=16, T; one CTA per head,
     # no segment scan) and, against KDA, at a shape where neither kernel segments (B=16, H=16, T=4096)
-    def time_calls(fn, n):
-        for _ in range(2):
-            fn()
-        barrier()
-        torch.cuda.synchronize()
-        start.record(stream)
-        for _ in range(n):
-            fn()
-        end.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(start.elapsed_time(end) / n)
 
     dp = synth.dplr_inputs(B=1, H=H_PREFILL, T=T, s0_std=0.02, seed=cfg["seed"] + 11, device=dev)
     dargs = [dp[n] for n in ("q", "k", "v", "a", "b", "g", "beta")]
@@ -356,21 +390,7 @@ def run_ours(args):
     del bw, bdo, bws
     assert kda.device_status() == 0
 
-    # the KDA layer: d_model=2048, H=16, rank 128, 65536 packed tokens in 8 sequences, random-init weights
-    lc = synth.LAYER_65K
-    lx, lW, lcu = synth.layer_inputs(d_model=lc["d_model"], H=lc["H"], Ttot=lc["Ttot"], nseq=lc["nseq"],
-                                     rank=lc["rank"], seed=lc["seed"] + rank, device=dev)
-    lpk = kda.pack_layer_weights(lW)
-    lcu_d = torch.tensor(lcu, dtype=torch.int32, device=dev)
-    ly = torch.empty_like(lx)
-    lfs = torch.empty((lc["nseq"], lc["H"], D, D), device=dev, dtype=torch.float32)
-    lws = torch.empty(kda.layer_fwd_workspace_bytes(lc["Ttot"], lc["d_model"], lc["H"], lc["rank"], lc["nseq"]),
-                      device=dev, dtype=torch.uint8)
-    layer_ms = time_calls(lambda: kda.layer_fwd(lx, lpk, lcu_d, out=ly, final_state=lfs, workspace=lws), 5)
-    HDl, dm, rk = lc["H"] * D, lc["d_model"], lc["rank"]
-    gemm_flop = 2 * lc["Ttot"] * (dm * (3 * HDl + 2 * rk + lc["H"]) + 2 * rk * HDl + HDl * dm)
-    layer_flop = gemm_flop + FLOP_PER_TOKEN_HEAD * lc["Ttot"] * lc["H"]
-    del lx, lW, lpk, ly, lfs, lws
+    layer = time_layer(kda, synth, dev, rank, time_calls, tc_peak, world)
     assert kda.device_status() == 0
 
     # end to end through the public call with host buffers (pinned), copies inside the timed region
@@ -433,11 +453,7 @@ def run_ours(args):
                                            "dplr_over_kda": eq_dplr_ms / eq_kda_ms}},
             "backward": {"workload": "B=1 H=16 T=8192: dq, dk, dv, dg, dbeta, dS0 by recurrent reverse mode",
                          "ms_per_call": bwd_ms, "tokens_per_s": world * bT / (bwd_ms / 1e3)},
-            "layer": {"workload": "KDA layer d_model=2048 H=16 rank=128, 65536 packed tokens (8 sequences), "
-                                  "random-init bf16 weights", "ms_per_call": layer_ms,
-                      "tokens_per_s": world * lc["Ttot"] / (layer_ms / 1e3),
-                      "tflops": layer_flop / (layer_ms / 1e3) / 1e12, "gemm_tflop_per_call": gemm_flop / 1e12,
-                      "tensor_peak_tflops": tc_peak, "frac": layer_flop / (layer_ms / 1e3) / 1e12 / tc_peak},
+            "layer": layer,
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,
@@ -458,6 +474,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=T_PREFILL, help="prefill length (profiling runs use a smaller one)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and the CPU baseline")
+    ap.add_argument("--layer-only", action="store_true", help="time only the KDA layer (profiling runs)")
     ap.add_argument("--warmup-seconds", type=float, default=1.5, help="minimum warm-up time (clock sampling)")
     args = ap.parse_args()
     if args.warmup < 3:

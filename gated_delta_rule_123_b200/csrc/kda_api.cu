@@ -287,7 +287,8 @@ static int check_layer_weights(const kda_layer_weights* w) {
     if (w->d_model % 8 || w->rank % 8) return fail(KDA_ERR_UNSUPPORTED, "d_model and rank must be multiples of 8");
     if (!w->W_in || !w->W_aup || !w->W_gup || !w->conv_w || !w->norm_w || !w->W_o)
         return fail(KDA_ERR_INVALID_ARG, "NULL weight pointer");
-    if (!aligned16(w->W_in) || !aligned16(w->W_aup) || !aligned16(w->W_gup) || !aligned16(w->W_o))
+    if (!aligned16(w->W_in) || !aligned16(w->W_aup) || !aligned16(w->W_gup) || !aligned16(w->W_o) ||
+        !aligned16(w->conv_w))
         return fail(KDA_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
     return KDA_OK;
 }

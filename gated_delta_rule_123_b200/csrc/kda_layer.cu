@@ -47,54 +47,102 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int nseq, int seq_len, 
 }
 __device__ __forceinline__ int seq_begin(const int32_t* cu, int seq_len, int n) { return cu ? cu[n] : n * seq_len; }
 
-// One warp per (token, head, tensor in {q,k,v}); lane owns 4 channels.  Taps
-// before the sequence's first token in this call read the cached history
-// conv_in [nseq][3][3 H 128] (row 2 = the token just before), or zero.
-__global__ void conv_silu_norm_kernel(const __nv_bfloat16* __restrict__ z, int ldz,
-                                      const __nv_bfloat16* __restrict__ conv_w, const int32_t* __restrict__ cu,
-                                      int nseq, int seq_len, int ntok, int H,
-                                      const __nv_bfloat16* __restrict__ conv_in, __nv_bfloat16* __restrict__ q,
-                                      __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v) {
-    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    const long long total = (long long)ntok * H * 3;
-    if (wid >= total) return;
-    const int which = int(wid % 3);
-    const int h = int((wid / 3) % H);
-    const int t = int(wid / (3LL * H));
-    const int n = seq_of(cu, nseq, seq_len, t);
-    const int s0 = seq_begin(cu, seq_len, n);
-    const int HD = H * kD;
-    const int col0 = which * HD + h * kD + lane * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int tt = t - 3 + j;
-        if (tt < s0 && !conv_in) continue;
-        const __nv_bfloat16* src = tt >= s0 ? z + (size_t)tt * ldz + col0
-                                            : conv_in + ((size_t)n * 3 + (3 + tt - s0)) * (3 * HD) + col0;
-        const uint2 raw = *reinterpret_cast<const uint2*>(src);
-        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        const float xv[4] = {__low2float(pr[0]), __high2float(pr[0]), __low2float(pr[1]), __high2float(pr[1])};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] += __bfloat162float(conv_w[(size_t)(col0 + u) * 4 + j]) * xv[u];
-    }
-    float ss = 0.f;
+// ShortConv + SiLU (+ L2 norm of q and k per head).  A CTA of 256 threads runs
+// one tensor (blockIdx.y: q, k or v) over kConvTok consecutive tokens and 2048
+// of its channels (blockIdx.z); thread i owns channels [8i, 8i + 8) of that
+// block (its 4 taps stay in registers), and a head's 128 channels are one
+// half-warp.  The last three inputs of each
+// channel are kept in registers as the window slides over the tokens, so every
+// projection row is read once; at a sequence start the window restarts from the
+// cached history conv_in [nseq][3][3 H 128] (row 2 = the token just before) or
+// from zero.  Loads and stores are 16 bytes.
+constexpr int kConvTok = 16;
+
+__device__ __forceinline__ void unpack8(const uint4& r, float* f) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        acc[u] = acc[u] / (1.f + __expf(-acc[u]));  // SiLU
-        ss += acc[u] * acc[u];
+        f[2 * u] = __low2float(p[u]);
+        f[2 * u + 1] = __high2float(p[u]);
     }
-    if (which < 2) {
+}
+
+__global__ void __launch_bounds__(256) conv_silu_norm_kernel(
+    const __nv_bfloat16* __restrict__ z, int ldz, const __nv_bfloat16* __restrict__ conv_w,
+    const int32_t* __restrict__ cu, int nseq, int seq_len, int ntok, int H, const __nv_bfloat16* __restrict__ conv_in,
+    __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v) {
+    const int HD = H * kD;
+    const int which = blockIdx.y;
+    const int c0 = (blockIdx.z * 256 + threadIdx.x) * 8;  // channel inside the tensor
+    if (c0 >= HD) return;  // whole half-warps (heads) drop out together
+    const unsigned hmask = 0xffffu << (threadIdx.x & 16);  // this half-warp
+    const int col = which * HD + c0;  // column of z and of the conv taps
+    const int t0 = blockIdx.x * kConvTok, t1 = min(ntok, t0 + kConvTok);
+    float w[8][4];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float f = rsqrtf(ss + 1e-6f);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] *= f;
+    for (int u = 0; u < 8; ++u) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(conv_w + (size_t)(col + u) * 4);
+        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        w[u][0] = __low2float(pr[0]);
+        w[u][1] = __high2float(pr[0]);
+        w[u][2] = __low2float(pr[1]);
+        w[u][3] = __high2float(pr[1]);
     }
     __nv_bfloat16* dst = which == 0 ? q : (which == 1 ? k : v);
-    __nv_bfloat162 o2[2] = {__floats2bfloat162_rn(acc[0], acc[1]), __floats2bfloat162_rn(acc[2], acc[3])};
-    *reinterpret_cast<uint2*>(dst + ((size_t)t * H + h) * kD + lane * 4) = *reinterpret_cast<uint2*>(o2);
+    int n = seq_of(cu, nseq, seq_len, t0);
+    int s_beg = seq_begin(cu, seq_len, n), s_end = seq_begin(cu, seq_len, n + 1);
+    float hist[3][8];  // inputs at t-3, t-2, t-1
+    auto load_hist = [&](int t) {  // window for token t, which starts at or after s_beg
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int tt = t - 3 + j;
+            if (tt >= s_beg) {
+                unpack8(*reinterpret_cast<const uint4*>(z + (size_t)tt * ldz + col), hist[j]);
+            } else if (conv_in) {
+                unpack8(*reinterpret_cast<const uint4*>(conv_in + ((size_t)n * 3 + (3 + tt - s_beg)) * (3 * HD) + col),
+                        hist[j]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) hist[j][u] = 0.f;
+            }
+        }
+    };
+    load_hist(t0);
+#pragma unroll 1
+    for (int t = t0; t < t1; ++t) {
+        while (t >= s_end) {  // a new sequence starts at t (empty ones are skipped)
+            ++n;
+            s_beg = s_end;
+            s_end = seq_begin(cu, seq_len, n + 1);
+            load_hist(t);
+        }
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4*>(z + (size_t)t * ldz + col), x);
+        float acc[8], ss = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float a = w[u][0] * hist[0][u] + w[u][1] * hist[1][u] + w[u][2] * hist[2][u] + w[u][3] * x[u];
+            a = a / (1.f + __expf(-a));  // SiLU
+            acc[u] = a;
+            ss += a * a;
+            hist[0][u] = hist[1][u];
+            hist[1][u] = hist[2][u];
+            hist[2][u] = x[u];
+        }
+        if (which < 2) {  // L2 norm over the head's 128 channels = this half-warp
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(hmask, ss, off);
+            const float f = rsqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] *= f;
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(dst + (size_t)t * HD + c0) = o;
+    }
 }
 
 // conv_out[n] = the last 3 conv inputs (q, k, v pre-activations) up to the end of
@@ -285,10 +333,10 @@ static int layer_pipeline(const void* x, const kda_layer_weights* w, const int32
         return KDA_ERR_CUDA;
     }
     {
-        const long long warps = (long long)ntok * H * 3;
-        conv_silu_norm_kernel<<<unsigned((warps + 7) / 8), 256, 0, stream>>>(
-            zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu, nseq, seq_len, ntok, H,
-            static_cast<const __nv_bfloat16*>(conv_in), q, k, v);
+        const dim3 grid(unsigned((ntok + kConvTok - 1) / kConvTok), 3, unsigned((HD + 2047) / 2048));
+        conv_silu_norm_kernel<<<grid, 256, 0, stream>>>(zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu,
+                                                        nseq, seq_len, ntok, H,
+                                                        static_cast<const __nv_bfloat16*>(conv_in), q, k, v);
     }
     if (conv_out) {
         const long long n = (long long)nseq * 3 * HD;

@@ -67,3 +67,10 @@ def test_layer_full_size_sampled_sequences(kda):
                      seed=cfg["seed"], check_seqs=pick)
     for ey, es in errs:
         assert ey < TOL_Y and es < TOL_S, errs
+
+
+def test_layer_more_than_16_heads(kda):
+    """H=20: the ShortConv kernel covers a tensor's channels in blocks of 2048."""
+    errs = run_layer(kda, d_model=256, H=20, Ttot=150, nseq=2, rank=32, seed=23)
+    for ey, es in errs:
+        assert ey < TOL_Y and es < TOL_S, errs
