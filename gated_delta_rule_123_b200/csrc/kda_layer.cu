@@ -55,8 +55,10 @@ __device__ __forceinline__ int seq_begin(const int32_t* cu, int seq_len, int n) 
 // channel are kept in registers as the window slides over the tokens, so every
 // projection row is read once; at a sequence start the window restarts from the
 // cached history conv_in [nseq][3][3 H 128] (row 2 = the token just before) or
-// from zero.  Loads and stores are 16 bytes.
-constexpr int kConvTok = 16;
+// from zero.  Loads and stores are 16 bytes, and all of a block's rows are
+// requested before the first is used (the kernel is bound by memory latency
+// otherwise).
+constexpr int kConvTok = 8;
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
@@ -107,9 +109,15 @@ __global__ void __launch_bounds__(256) conv_silu_norm_kernel(
             }
         }
     };
+    uint4 rows[kConvTok];
+#pragma unroll
+    for (int j = 0; j < kConvTok; ++j)
+        if (t0 + j < t1) rows[j] = *reinterpret_cast<const uint4*>(z + (size_t)(t0 + j) * ldz + col);
     load_hist(t0);
-#pragma unroll 1
-    for (int t = t0; t < t1; ++t) {
+#pragma unroll
+    for (int j = 0; j < kConvTok; ++j) {
+        const int t = t0 + j;
+        if (t >= t1) break;
         while (t >= s_end) {  // a new sequence starts at t (empty ones are skipped)
             ++n;
             s_beg = s_end;
@@ -117,12 +125,12 @@ __global__ void __launch_bounds__(256) conv_silu_norm_kernel(
             load_hist(t);
         }
         float x[8];
-        unpack8(*reinterpret_cast<const uint4*>(z + (size_t)t * ldz + col), x);
+        unpack8(rows[j], x);
         float acc[8], ss = 0.f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             float a = w[u][0] * hist[0][u] + w[u][1] * hist[1][u] + w[u][2] * hist[2][u] + w[u][3] * x[u];
-            a = a / (1.f + __expf(-a));  // SiLU
+            a = __fdividef(a, 1.f + __expf(-a));  // SiLU
             acc[u] = a;
             ss += a * a;
             hist[0][u] = hist[1][u];
