@@ -2,8 +2,8 @@
 """KDA on B200: prefill tokens/s at B=1, H=16, T=65536 and decode state GB/s.
 
 One step = one ``kda_chunk_fwd`` call over a B=1, H=16, T=65536, d=128 bf16
-sequence with a random fp32 initial state (plan + segment summary + combine +
-output kernels).  The decode figure is measured in the same run on the
+sequence with a random fp32 initial state (plan; first segment's output with the
+later segments' maps; combine; the later segments' outputs).  The decode figure is measured in the same run on the
 B=256, H=32 decode workload (512 MiB fp32 state updated in place).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -276,16 +276,21 @@ def run_ours(args):
     assert kda.device_status() == 0
     value = world * T / (ms / 1e3)
 
-    # roofline of the dominant kernel (the output pass): algorithmic bytes per launch / its time
-    alg_bytes = BYTES_PER_TOKEN_HEAD * T * H_PREFILL
+    # roofline of the output launch (the later segments' outputs; everything when unsegmented):
+    # algorithmic bytes of the tokens it processes / its time
+    seg_tok = int(kda.lib().kda_chunk_fwd_segment_tokens(1, T, H_PREFILL, 0))
+    out_tokens = T - min(seg_tok, T)
+    alg_bytes = BYTES_PER_TOKEN_HEAD * out_tokens * H_PREFILL
     achieved = alg_bytes / (out_ms / 1e3) / 1e9
     traffic = profiled_traffic("chunk_output_T65536_traffic.md", "gated_delta_rule_123_b200/csrc/kda_chunk.cu")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic if T == T_PREFILL else None,
-                "traffic_unit": "bytes per launch", "algorithmic_bytes": alg_bytes, "kernel": "chunk_kernel<output>",
-                "peak_kind": peak_kind,
-                "step_frac": alg_bytes / (ms / 1e3) / 1e9 / hbm_peak,
-                "kernel_ms": {"plan": plan_ms, "summary": sum_ms, "combine": comb_ms, "output": out_ms},
+                "traffic_unit": "bytes per launch", "algorithmic_bytes": alg_bytes,
+                "kernel": "chunk_phase2_kernel (outputs of segments 1..G-1)", "tokens_per_launch": out_tokens * H_PREFILL,
+                "segment_tokens": seg_tok, "peak_kind": peak_kind,
+                "step_frac": BYTES_PER_TOKEN_HEAD * T * H_PREFILL / (ms / 1e3) / 1e9 / hbm_peak,
+                "kernel_ms": {"plan": plan_ms, "first_segment_and_maps": sum_ms, "combine": comb_ms,
+                              "later_segments": out_ms},
                 "tensor_tflops_step": FLOP_PER_TOKEN_HEAD * T * H_PREFILL / (ms / 1e3) / 1e12,
                 "tensor_peak": tc_peak}
 

@@ -28,6 +28,7 @@ SYMBOLS = (
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
     "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
+    "kda_chunk_fwd_segment_tokens",
 )
 
 
@@ -56,6 +57,8 @@ def _load():
     lib.kda_device_status.restype = i
     lib.kda_chunk_fwd_workspace.argtypes = [i, i, i, i, i, i]
     lib.kda_chunk_fwd_workspace.restype = sz
+    lib.kda_chunk_fwd_segment_tokens.argtypes = [i, i, i, i]
+    lib.kda_chunk_fwd_segment_tokens.restype = i
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i
     lib.kda_gdn_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]

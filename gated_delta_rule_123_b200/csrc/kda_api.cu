@@ -17,6 +17,7 @@ int launch_recurrent_bwd(const void* q, const void* k, const void* v, const floa
                          const float* init, const void* dout, const float* dfinal, float* dq, float* dk, float* dv,
                          float* dg, float* dbeta, float* dinit, int B, int Tn, int H, int dtype, float scale,
                          void* ws, size_t ws_bytes, cudaStream_t stream, const char** why);
+int chunk_segment_tokens(int B, int T, int H, int num_seqs);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
                          cudaStream_t stream);
@@ -87,6 +88,11 @@ int kda_device_status(void* stream) {
         return fail(KDA_ERR_TIMEOUT, msg);
     }
     return KDA_OK;
+}
+
+int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs) {
+    if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;
+    return chunk_segment_tokens(B, T, H, num_seqs);
 }
 
 size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk) {

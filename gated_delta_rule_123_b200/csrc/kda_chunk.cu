@@ -122,7 +122,7 @@ struct ChunkArgs {
     const int* n_items;
     float* segN;
     float* segX;
-    const float* segS;
+    float* segS;  // per-segment start states (phase 1 writes segment 1's, the combine pass the rest)
     int H;
     float scale;
 };
@@ -174,16 +174,20 @@ constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
 
 // kSummary = true : segment summary (zero start state, identity X, no output).
-// kSummary = false: output pass from the segment's true start state.
+// kSummary = false: output from the segment's true start state (the initial state
+//                   for segment 0, the combine pass's result for the others).
+// A segmented sequence runs in two phases of launches: phase 1 computes the
+// output of segment 0 (whose start state is known) side by side with the maps of
+// segments 1..G-2; after the combine pass, phase 2 computes the outputs of
+// segments 1..G-1.  Both phases keep G-1 CTAs per (sequence, head) busy.
 // kScalarGate = true: one log-gate per (token, head) (gated DeltaNet); every key
 // channel shares it, so the decay factors are per row instead of per element.
 constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
 
 template <bool kSummary, typename OutT, bool kScalarGate>
-__global__ void __launch_bounds__(kThreads, 1)
-    chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                 const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
+__device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                           const CUtensorMap& tm_g, const CUtensorMap& tm_o, const ChunkArgs& p,
+                                           const SegItem it) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw;
     const uint32_t sbase = smem_u32(sm);
@@ -196,9 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, part = warp >> 2;  // TMEM lane quadrant; column quarter
     const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
-    if (item_id >= *p.n_items) return;
-    const SegItem it = p.items[item_id];
-    if (kSummary && it.g == it.G - 1) return;  // the last segment's map is never needed
 
     float* sBeta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64] beta per chunk parity
     float* sFrOp = sBeta2 + 128;                               // [128] post(prev) * e^{mp}
@@ -277,9 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
         const float* src = nullptr;
         if (!kSummary) {
-            // A segmented sequence takes every start state (segment 0's too) from
-            // the combine pass, so final_state may alias initial_state.
-            if (it.G == 1)
+            // segment 0 starts from the initial state (read in phase 1, before any
+            // final state is written, so the two may alias); the others from the
+            // combine pass
+            if (it.g == 0)
                 src = p.init_state ? p.init_state + (size_t(it.seq) * H + h) * (kD * kD) : nullptr;
             else
                 src = p.segS + (size_t(item_id) * H + h) * (kD * kD);
@@ -1024,8 +1026,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kSummary) {
             dstS = p.segN + (size_t(item_id) * H + h) * (kD * kD);
             dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
-        } else if (it.g == it.G - 1 && p.final_state) {
-            dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
+        } else if (it.g == it.G - 1) {
+            if (p.final_state) dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
+        } else if (it.g == 0) {  // segment 1's start state, for the combine pass and phase 2
+            dstS = p.segS + (size_t(item_id + 1) * H + h) * (kD * kD);
         }
         tc_fence_after();
         auto store = [&](uint32_t tcol, float* dst) {
@@ -1072,6 +1076,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < 128) atomicAdd(&g_warp_cycles[(kSummary ? 128 : 0) + tid], s_warp_cyc[tid]);
 #endif
     if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// Phase 1 (and the only launch of an unsegmented call): segment 0's output, and
+// the maps of segments 1..G-2.
+template <typename OutT, bool kScalarGate>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_phase1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                        const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
+    if (int(blockIdx.x) >= *p.n_items) return;
+    const SegItem it = p.items[blockIdx.x];
+    if (it.g == 0)
+        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+    else if (it.g < it.G - 1)
+        chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+}
+
+// Phase 2: the outputs of segments 1..G-1 from the combine pass's start states.
+template <typename OutT, bool kScalarGate>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_phase2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                        const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
+    if (int(blockIdx.x) >= *p.n_items) return;
+    const SegItem it = p.items[blockIdx.x];
+    if (it.g >= 1) chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
 }
 
 // ---------------------------------------------------------------- plan
@@ -1139,7 +1169,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
     const int item = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
     if (item >= *n_items) return;
     const SegItem it = items[item];
-    if (it.g != 0 || it.G < 2) return;
+    if (it.g != 0 || it.G < 3) return;  // S_1 comes from phase 1; S_2.. are chained here
     extern __shared__ __align__(128) uint8_t csm[];
     float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
     float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
@@ -1154,28 +1184,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
         fence_mbar_init();
     }
     __syncthreads();
-    auto fetch = [&](int g) {
-        mbar_arrive_expect_tx(&bar[g & 1], 65536u);
-        bulk_load_1d(sX + (g & 1) * kD * kD, segXt + size_t(item + g) * H * (kD * kD) + hs, 65536u, &bar[g & 1]);
+    // step j = 0, 1, ... maps S_{j+1} to S_{j+2} with segment j+1's map
+    auto fetch = [&](int j) {
+        mbar_arrive_expect_tx(&bar[j & 1], 65536u);
+        bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + 1 + j) * H * (kD * kD) + hs, 65536u, &bar[j & 1]);
     };
     if (tid == 0) fetch(0);
+    (void)init;
     for (int e = tid; e < kD * kCombCols; e += 256) {
         const int kk = e / kCombCols, jj = e % kCombCols;
-        const float s0 = init ? init[size_t(it.seq) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] : 0.f;
-        sS[e] = s0;
-        segS[size_t(item) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] = s0;
+        sS[e] = segS[size_t(item + 1) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj];
     }
     __syncthreads();
     bool ok = true;
-    int fetched = 1, g = 0;  // fetches issued (thread 0) and the step being consumed
-    for (; g + 1 < it.G; ++g) {
-        if (tid == 0 && g + 2 < it.G) {
-            fetch(g + 1);
-            fetched = g + 2;
+    int fetched = 1, j = 0;  // fetches issued (thread 0) and the step being consumed
+    for (; j + 2 < it.G; ++j) {
+        const int g = j + 1;  // the segment whose map this step applies
+        if (tid == 0 && j + 3 < it.G) {
+            fetch(j + 1);
+            fetched = j + 2;
         }
-        ok = mbar_wait(&bar[g & 1], uint32_t((g >> 1) & 1), 8);
+        ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
         if (__syncthreads_or(!ok)) break;
-        const float* X = sX + (g & 1) * kD * kD;
+        const float* X = sX + (j & 1) * kD * kD;
         const size_t base = size_t(item + g) * H * (kD * kD) + hs;
         float acc[2][4];
 #pragma unroll
@@ -1201,7 +1232,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
         __syncthreads();
     }
     if (tid == 0 && !ok) {  // let copies still in flight land before the shared memory is released
-        for (int f = g; f < fetched; ++f) mbar_wait(&bar[f & 1], uint32_t((f >> 1) & 1), 8);
+        for (int f = j; f < fetched; ++f) mbar_wait(&bar[f & 1], uint32_t((f >> 1) & 1), 8);
     }
 }
 
@@ -1281,7 +1312,7 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     const long long pairs = (long long)pl.N * H;
     int L = 1 << 30;
     if (pairs > 0 && pairs * 3 <= nsm) {
-        const long long G = nsm / pairs;  // segments per sequence
+        const long long G = nsm / pairs + 1;  // segments per sequence: G-1 CTAs per pair in each phase
         const long long per_seq = (chunks_bound + pl.N - 1) / pl.N;
         L = int((per_seq + G - 1) / G);
         if (L < 1) L = 1;
@@ -1306,22 +1337,29 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     return pl;
 }
 
-template <bool S, typename O, bool G>
-static cudaError_t set_smem_attr() {
-    static bool done = false;
-    if (done) return cudaSuccess;
-    cudaError_t e =
-        cudaFuncSetAttribute(chunk_kernel<S, O, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) done = true;
-    return e;
+template <int kPhase, typename O, bool G>
+static int launch_phase(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a, cudaStream_t stream) {
+    auto kern = kPhase == 1 ? chunk_phase1_kernel<O, G> : chunk_phase2_kernel<O, G>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        attr = true;
+    }
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+    return KDA_OK;
 }
 
-template <bool S, typename O, bool G>
-static int launch_pass(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a, cudaStream_t stream) {
-    if (set_smem_attr<S, O, G>() != cudaSuccess) return KDA_ERR_CUDA;
-    chunk_kernel<S, O, G><<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
-    return KDA_OK;
+template <int kPhase>
+static int launch_phase_for(int dtype, int scalar_gate, dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk,
+                            const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a,
+                            cudaStream_t stream) {
+    if (dtype == KDA_FP32)
+        return scalar_gate ? launch_phase<kPhase, float, true>(grid, mq, mk, mv, mg, mo, a, stream)
+                           : launch_phase<kPhase, float, false>(grid, mq, mk, mv, mg, mo, a, stream);
+    return scalar_gate ? launch_phase<kPhase, __nv_bfloat16, true>(grid, mq, mk, mv, mg, mo, a, stream)
+                       : launch_phase<kPhase, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
 }
 
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -1395,14 +1433,17 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     a.n_items = n_items;
     a.segN = reinterpret_cast<float*>(w + pl.off_segN);
     a.segX = reinterpret_cast<float*>(w + pl.off_segX);
-    a.segS = reinterpret_cast<const float*>(w + pl.off_segS);
+    a.segS = reinterpret_cast<float*>(w + pl.off_segS);
     a.H = H;
     a.scale = scale;
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
+    if (!pl.scan && ev) {  // one launch: it is timed as the output pass
+        cudaEventRecord(ev[2], stream);
+        cudaEventRecord(ev[3], stream);
+    }
+    const int r1 = launch_phase_for<1>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
+    if (r1 != KDA_OK) return r1;
     if (pl.scan) {
-        const int rs = scalar_gate ? launch_pass<true, __nv_bfloat16, true>(grid, mq, mk, mv, mg, mo, a, stream)
-                                   : launch_pass<true, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
-        if (rs != KDA_OK) return rs;
         if (ev) cudaEventRecord(ev[2], stream);
         static bool comb_attr = false;
         if (!comb_attr) {
@@ -1414,18 +1455,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
             items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) cudaEventRecord(ev[3], stream);
-    } else if (ev) {
-        cudaEventRecord(ev[2], stream);
-        cudaEventRecord(ev[3], stream);
+        const int r2 = launch_phase_for<2>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
+        if (r2 != KDA_OK) return r2;
     }
-    int ro;
-    if (dtype == KDA_FP32)
-        ro = scalar_gate ? launch_pass<false, float, true>(grid, mq, mk, mv, mg, mo, a, stream)
-                         : launch_pass<false, float, false>(grid, mq, mk, mv, mg, mo, a, stream);
-    else
-        ro = scalar_gate ? launch_pass<false, __nv_bfloat16, true>(grid, mq, mk, mv, mg, mo, a, stream)
-                         : launch_pass<false, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
-    if (ro != KDA_OK) return ro;
     if (ev) cudaEventRecord(ev[4], stream);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -1453,6 +1485,11 @@ extern "C" int kda_debug_warp_cycles(unsigned long long* out, int reset) {
     return 0;
 }
 #endif
+
+int chunk_segment_tokens(int B, int T, int H, int num_seqs) {
+    const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count());
+    return pl.scan ? pl.L * kC : 0;
+}
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
     return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total;

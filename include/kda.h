@@ -76,10 +76,11 @@ int kda_device_status(void *stream);
 /* Optional tracing hook for kda_chunk_fwd.  When `events` is non-NULL it must
  * point to 5 cudaEvent_t created by the caller on the current device; every
  * later kda_chunk_fwd call on this thread records them on its stream around
- * its kernels: [0] before the plan kernel, [1] after it, [2] after the segment
- * summary pass (same as [1] when the sequence is not segmented), [3] after the
- * combine pass, [4] after the output pass.  Pass NULL to stop.  The events stay
- * owned by the caller. */
+ * its kernels: [0] before the plan kernel, [1] after it, [2] after the first
+ * phase (segment 0's output and the later segments' maps; same as [1] when the
+ * sequences are not segmented), [3] after the combine pass, [4] after the
+ * outputs of the later segments (or of everything, unsegmented).  Pass NULL to
+ * stop.  The events stay owned by the caller. */
 int kda_set_trace_events(void *events, int n_events);
 
 /* ------------------------------------------------------------------------
@@ -120,6 +121,13 @@ int kda_set_trace_events(void *events, int n_events);
  * accumulation; the state is carried in fp32.  fp32 inputs are rounded to
  * bf16 where they feed the tensor cores.
  */
+/* How a kda_chunk_fwd call with these sizes on the current device is split:
+ * 0 when every (sequence, head) runs in one CTA; otherwise the segment length
+ * in tokens.  A segmented call runs its first segment and the segment maps in
+ * one launch, then the combine pass, then the outputs of the later segments.
+ * Informational (profiling); the result never changes what is computed. */
+int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs);
+
 /* Workspace bytes for a kda_chunk_fwd call with the same B, T, H, num_seqs
  * (0 = dense), dtype and l2norm_qk, on the current device. */
 size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk);
