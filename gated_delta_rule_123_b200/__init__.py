@@ -28,7 +28,7 @@ SYMBOLS = (
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
     "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
-    "kda_chunk_fwd_segment_tokens",
+    "kda_chunk_fwd_segment_tokens", "kda_chunk_fwd_workspace_min",
 )
 
 
@@ -57,6 +57,8 @@ def _load():
     lib.kda_device_status.restype = i
     lib.kda_chunk_fwd_workspace.argtypes = [i, i, i, i, i, i]
     lib.kda_chunk_fwd_workspace.restype = sz
+    lib.kda_chunk_fwd_workspace_min.argtypes = [i, i, i, i, i, i]
+    lib.kda_chunk_fwd_workspace_min.restype = sz
     lib.kda_chunk_fwd_segment_tokens.argtypes = [i, i, i, i]
     lib.kda_chunk_fwd_segment_tokens.restype = i
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
@@ -177,9 +179,13 @@ def _chunk_call(fn, name, q, k, v, g, beta, initial_state, cu_seqlens, scale, l2
     fs = final_state
     if fs is None and output_final_state:
         fs = torch.empty((N, H, D, D), device=q.device, dtype=torch.float32)
-    wsz = chunk_fwd_workspace_bytes(B, T, H, nseq, dt, l2norm_qk)
-    if workspace is None or workspace.numel() < wsz:
-        workspace = torch.empty(max(wsz, 1), device=q.device, dtype=torch.uint8)
+    # a caller's workspace is used as is if it has at least the minimal size (the library
+    # then picks the schedule that fits); otherwise one of the full size is allocated
+    wmin = int(_lib.kda_chunk_fwd_workspace_min(B, T, H, nseq, dt, int(l2norm_qk)))
+    if workspace is None or workspace.numel() < wmin:
+        workspace = torch.empty(max(chunk_fwd_workspace_bytes(B, T, H, nseq, dt, l2norm_qk), 1), device=q.device,
+                                dtype=torch.uint8)
+    wsz = workspace.numel()
     rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(fs), _ptr(o),
             _ptr(cu_seqlens), nseq, B, T, H, dt, float(scale), int(l2norm_qk), _ptr(workspace), wsz,
             _stream(q.device))

@@ -39,6 +39,8 @@
 //    affine map S_end = X S_start + N (X carried like a second state with
 //    U = 0), a short combine pass chains the maps, and the output pass runs
 //    every segment from its true start state.  Only the state crosses chunks.
+#include <cmath>
+
 #include <cub/block/block_scan.cuh>
 
 #include "kda_common.cuh"
@@ -112,8 +114,20 @@ static_assert(kSmemBytes <= 232448, "shared memory plan");
 // [U|O] and [O|S] are contiguous so one N=128 and one N=192 MMA can fill them.
 constexpr uint32_t TM_U = 0, TM_O = 64, TM_S = 128, TM_AP = 256, TM_W = 320, TM_X = 384;
 
+// Per-chunk products of a segment's map pass, reused by its output pass: one
+// image per (segment item, chunk, head), laid out as the output kernel's tiles
+// so that it loads straight into MMA operands: -W^T | Qp (adjacent: one N=128
+// operand), T beta, P | Km (adjacent: one N=192 operand), then the chunk's
+// frame factors post(prev) e^{mp}, post(prev) e^{mk}, e^{b_C - mk} (fp32 [3][128]).
+constexpr uint32_t PI_WN = 0, PI_QP = 16384, PI_TB = 32768, PI_P = 40960, PI_KM = 49152, PI_FR = 65536;
+constexpr uint32_t kProdBytes = 67584;
+static_assert(PI_QP - PI_WN == OFF_QP - OFF_WN && PI_KM - PI_P == OFF_KM - OFF_P && PI_P - PI_TB == OFF_P - OFF_TB,
+              "product image keeps the operand stacks");
+
 struct ChunkArgs {
     const float* beta;
+    uint8_t* prod;    // product images [item][prodL][H] (segmented calls)
+    int prodL;        // chunk slots per item
     const float* gs;  // per-head scalar log-gates [Ttot][H] (scalar-gate kernels only)
     const float* init_state;
     float* final_state;
@@ -158,6 +172,19 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t s
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Global -> shared bulk copy completing on an mbarrier (16-byte aligned addresses and size).
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Shared -> global bulk copy (16-byte aligned addresses and size), in the current bulk group.
+__device__ __forceinline__ void bulk_store_1d(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -216,7 +243,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     // W^T spill: fp32 A over U~^T, fp32 T over -W^T.
     float* sA = reinterpret_cast<float*>(sm + OFF_UT);
     float* sT = reinterpret_cast<float*>(sm + OFF_WN);
-    constexpr int kLoader = 96;  // the thread that issues every TMA load (warp 3, lane 0)
+    constexpr int kLoader = 96;    // the thread that issues every TMA load (warp 3, lane 0)
+    constexpr int kExporter = 32;  // the thread that issues the map pass's product exports (warp 1)
 
     if (warp == 0) {
         tmem_alloc(sTmem, 512);
@@ -229,7 +257,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         fence_mbar_init();
     }
     if (tid == 64) {
-        if (!kSummary) prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         if (!kScalarGate) prefetch_tmap(&tm_g);
@@ -252,11 +280,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 
     auto issue_qkg = [&](int c) {
         const int t0 = t_begin + c * kC;
-        mbar_arrive_expect_tx(&bars[0], (kSummary ? 49152u : 65536u) - (kScalarGate ? 32768u : 0u));
-        if (!kSummary) {
-            tma_load_3d(sm + OFF_Q, &tm_q, &bars[0], 0, h, t0);
-            tma_load_3d(sm + OFF_Q + 8192, &tm_q, &bars[0], 64, h, t0);
-        }
+        mbar_arrive_expect_tx(&bars[0], 65536u - (kScalarGate ? 32768u : 0u));
+        tma_load_3d(sm + OFF_Q, &tm_q, &bars[0], 0, h, t0);
+        tma_load_3d(sm + OFF_Q + 8192, &tm_q, &bars[0], 64, h, t0);
         tma_load_3d(sm + OFF_K, &tm_k, &bars[0], 0, h, t0);
         tma_load_3d(sm + OFF_K + 8192, &tm_k, &bars[0], 64, h, t0);
         if (!kScalarGate) tma_load_3d(sm + OFF_G, &tm_g, &bars[0], 0, h, t0);
@@ -319,8 +345,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // U~^T (K) x Km (K)
     const uint32_t id_so2 = idesc_bf16(128, 128, 0, 1); // S'^T (K) x [-W^T | Qp] (MN)
     const uint32_t id_os = idesc_bf16(128, 192, 0, 0);  // U~^T (K) x [P^T | Km] (K)
-    // Summary pass: X'^T operand halves over the unused q / Qp tiles, U_X~^T over T beta + P.
-    const uint32_t XT0 = kSummary ? OFF_Q : 0, XT1 = kSummary ? OFF_QP : 0, UXT = OFF_TB;
+    // Summary pass: X'^T in TMEM over the [A;P] columns once they are read out (A operand of
+    // the U_X~ MMA); U_X~^T over T beta + P once both are exported.
+    const uint32_t UXT = OFF_TB;
+    const uint32_t TM_XP = TM_AP;
 
     // ---- gated operands of a chunk.  Chunk c+1's are built while chunk c's last
     // tensor-core MMAs run, in pieces placed by which tiles those MMAs still read:
@@ -352,7 +380,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 if (w < 16) {
                     const int box = w >> 3, j = w & 7;
                     st_shared_v4(sbase + OFF_K + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
-                    if (!kSummary) st_shared_v4(sbase + OFF_Q + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
+                    st_shared_v4(sbase + OFF_Q + box * 8192 + r * 128 + j * 16, 0u, 0u, 0u, 0u);
                 }
             }
             __syncthreads();
@@ -428,7 +456,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 const int j = h8 * 8 + e + u, r = rq * 16 + j;
                 const uint32_t off = e_box + sw128_off(r, ch & 63);
                 kv[u] = bf16_at(sKb, off);
-                qv[u] = kSummary ? 0.f : (unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc);
+                qv[u] = unit_scale ? bf16_at(sQb, off) : bf16_at(sQb, off) * sc;
                 if (factored && kScalarGate) {  // per-row factors, shared by every channel
                     e1[u] = sFac[r];
                     e2[u] = sFac[64 + r];
@@ -451,9 +479,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         const int j8 = (rq * 16 + h8 * 8) >> 3;
         st_shared_v4(sbase + OFF_KP + sw128_chunk(ch, j8), opk[h8 * 4], opk[h8 * 4 + 1], opk[h8 * 4 + 2],
                      opk[h8 * 4 + 3]);
-        if (!kSummary)
-            st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), opq[h8 * 4], opq[h8 * 4 + 1], opq[h8 * 4 + 2],
-                         opq[h8 * 4 + 3]);
+        st_shared_v4(sbase + OFF_QP + sw128_chunk(ch, j8), opq[h8 * 4], opq[h8 * 4 + 1], opq[h8 * 4 + 2],
+                     opq[h8 * 4 + 3]);
     };
     auto e_put_m = [&]() {
 #pragma unroll
@@ -550,13 +577,28 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         long long ts_ = clock64(), tw0_ = ts_;
 #endif
         KDA_STAGE(1);
+        // the map pass exports what the output pass of this segment reuses
+        uint8_t* img = (kSummary && p.prod) ? p.prod + ((size_t(item_id) * p.prodL + c) * H + h) * kProdBytes : nullptr;
+        if (img) {
+            if (tid == kExporter) {  // Qp and Km of this chunk are final (built before the last barrier)
+                bulk_store_1d(img + PI_QP, sm + OFF_QP, 16384u);
+                bulk_store_1d(img + PI_KM, sm + OFF_KM, 16384u);
+                bulk_commit();
+            }
+            if (tid < 128) {
+                float* fr = reinterpret_cast<float*>(img + PI_FR);
+                fr[tid] = sFrOp[tid];
+                fr[128 + tid] = sFrAcc[tid];
+                fr[256 + tid] = sPost[(c & 1) * 128 + tid];
+            }
+        }
 
         // ===== A (scaled by beta, strictly lower) and P (lower incl. diagonal) =====
         if (fast && tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, kSummary ? 0u : OFF_QP - OFF_KP, 1024);
+                const uint64_t a = sdesc_sw128(sbase + OFF_KP + ks * 2048, OFF_QP - OFF_KP, 1024);
                 const uint64_t b = sdesc_sw128(sbase + OFF_KM + ks * 2048, 8192, 1024);
                 umma_bf16(tbase + TM_AP, a, b, id_ap, ks > 0);
             }
@@ -594,9 +636,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 for (int cb = 0; cb < 2; ++cb) tmem_st16(tbase + tcol + lane_off + part * 32 + cb * 16, x + cb * 16);
             };
             frame(TM_S, OFF_ST, OFF_ST + 16384);
-            if (kSummary) {
-                frame(TM_X, XT0, XT1);
-            } else {  // O^T starts at zero: the merged [U~|O] MMA below accumulates into both halves
+            if (!kSummary) {  // O^T starts at zero: the merged [U~|O] MMA below accumulates into both halves
                 float z[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) z[j] = 0.f;
@@ -604,7 +644,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             }
             tmem_wait_st();
         }
-        if (!kSummary && tid == 0) bulk_wait_read0();  // the previous O tile (over U~^T / sA) is read out
+        // the previous O tile (over U~^T / sA) and the previous chunk's exported -W^T (under T)
+        // have been read out
+        if (tid == 0 || (kSummary && tid == kExporter)) bulk_wait_read0();
         if (fast) {
             ok = mbar_wait(&bars[2], ph_mma, 2);
             ph_mma ^= 1;
@@ -638,7 +680,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                     w4.w = (i + 3 < vrow) ? br * vals[j + 3] : 0.f;
                     *reinterpret_cast<float4*>(&sA[sidx(vrow, i)]) = w4;
                 }
-            } else if (!kSummary) {
+            } else {
                 const int r = vrow - 64;
 #pragma unroll
                 for (int q4 = 0; q4 < 2; ++q4) {
@@ -675,7 +717,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                         const uint32_t offi = uint32_t(cc >> 6) * 8192u + sw128_off(i, cc & 63);
                         const float ki = bf16_at(sKb, offi) * f;
                         ra[u] += bf16_at(sKb, offr) * ki;
-                        if (!kSummary) rp[u] += bf16_at(sQb, offr) * ki;
+                        rp[u] += bf16_at(sQb, offr) * ki;
                     }
                 }
             }
@@ -685,8 +727,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 pend_qkg = true;
             }
             for (int e = tid; e < 64 * 64; e += kThreads) sA[e] = 0.f;
-            if (!kSummary)
-                for (int e = tid; e < 512; e += kThreads) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
+            for (int e = tid; e < 512; e += kThreads) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
             __syncthreads();
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
@@ -697,15 +738,40 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
                 const int i = pidx - r * (r + 1) / 2;
                 if (i < r) sA[((r >> 4) == (i >> 4)) ? sidx(i, r) : sidx(r, i)] = sBeta[r] * ra[u];
-                if (!kSummary)
-                    *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) =
-                        __float2bfloat16_rn(rp[u] * p.scale);
+                *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) = __float2bfloat16_rn(rp[u] * p.scale);
             }
         }
         KDA_WMARK(0);
+        tc_fence_before();
         __syncthreads();
+        tc_fence_after();
         KDA_WMARK(1);
         KDA_STAGE(3);
+        if (kSummary && warp >= 4) {
+            // X' = X e^{mp} as bf16 pairs into the [A;P] columns (read out by now): the A operand
+            // of the U_X~ MMA; TMEM X <- X e^{mk}.  Warps 4..15 do it while warps 0..3 run the
+            // diagonal UT solves: the three warps of a TMEM lane quadrant take key columns
+            // [0, 64), [64, 96) and [96, 128).
+            const int slot = (warp >> 2) - 1;
+            for (int kb = slot == 0 ? 0 : 32 * (slot + 1); kb < (slot == 0 ? 64 : 32 * (slot + 2)); kb += 32) {
+                float x[32];
+                tmem_ld16(tbase + TM_X + lane_off + kb, x);
+                tmem_ld16(tbase + TM_X + lane_off + kb + 16, x + 16);
+                tmem_wait_ld();
+                float xp[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const int k0 = kb + j;
+                    xp[j >> 1] = __uint_as_float(pack_bf16x2(x[j] * sFrOp[k0], x[j + 1] * sFrOp[k0 + 1]));
+                    x[j] *= sFrAcc[k0];
+                    x[j + 1] *= sFrAcc[k0 + 1];
+                }
+                tmem_st16(tbase + TM_X + lane_off + kb, x);
+                tmem_st16(tbase + TM_X + lane_off + kb + 16, x + 16);
+                tmem_st16(tbase + TM_XP + lane_off + kb / 2, xp);
+            }
+            tmem_wait_st();
+        }
 
         // ===== UT transform: T = (I + A)^{-1}, blocked forward substitution =====
         if (warp < 4 && lane < 16) {
@@ -849,6 +915,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         ph_v ^= 1;
         if (tid == kLoader) pend_v = false;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        if (img && tid == kExporter) {  // T beta and P (adjacent tiles) are final
+            bulk_store_1d(img + PI_TB, sm + OFF_TB, 16384u);
+            bulk_commit();
+        }
         KDA_STAGE(6);
 
         // ===== W^T = Kp^T (T beta)^T and U^T = V^T (T beta)^T =====
@@ -886,6 +956,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (img && tid == kExporter) {  // -W^T is final
+            bulk_store_1d(img + PI_WN, sm + OFF_WN, 16384u);
+            bulk_commit();
+        }
 
         KDA_STAGE(9);
         // ===== U~^T = U^T - S'^T W^T ;  O^T = S'^T Qp  (or U_X~^T = -X'^T W^T) =====
@@ -900,8 +974,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                               id_so2, 1);
                 } else {
                     umma_bf16(tbase + TM_U, a, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, 1);
-                    const uint64_t ax = sdesc_sw128(sbase + ((ks >> 2) ? XT1 : XT0) + (ks & 3) * 32, 16, 1024);
-                    umma_bf16(tbase + TM_O, ax, sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, ks > 0);
+                    umma_bf16_tmem_a(tbase + TM_O, tbase + TM_XP + ks * 8,
+                                     sdesc_sw128(sbase + OFF_WN + ks * 2048, 8192, 1024), id_so, ks > 0);
                 }
             }
             umma_commit(&bars[2]);
@@ -921,6 +995,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         ok = mbar_wait(&bars[2], ph_mma, 5);
         ph_mma ^= 1;
         tc_fence_after();
+        // the exports have read Qp (rewritten next) and T beta + P (U_X~^T goes over them)
+        if (img && tid == kExporter) bulk_wait_read0();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(10);
         if (has_next) {  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
@@ -1067,7 +1143,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         }
         if (tid == 0) mbar_wait(&bars[2], ph_mma, 7);
     }
-    if (!kSummary && tid == 0) bulk_wait0();
+    if (tid == 0 || tid == kExporter) bulk_wait0();  // O tiles and exported products are written
     if (tid < 64) cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -1076,6 +1152,229 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     if (tid < 128) atomicAdd(&g_warp_cycles[(kSummary ? 128 : 0) + tid], s_warp_cyc[tid]);
 #endif
     if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// Output pass of a segment whose map pass exported its per-chunk products: per
+// chunk it loads the product image (double-buffered, one bulk copy) and V, and
+// runs only the state chain -- the frame pass, U^T = V^T (T beta)^T followed by
+// [U~ | O] += S'^T [-W^T | Qp] in one MMA group, the U~ spill, [O | S] +=
+// U~^T [P | Km], and the O store.  The segment's end state is not needed (the
+// combine pass produced the next segment's start state).
+namespace light {
+constexpr uint32_t PROD = 0;                          // 2 product images
+constexpr uint32_t V = 2 * kProdBytes;                // 2 x [64 tok][128 v]
+constexpr uint32_t ST = V + 32768;                    // S'^T, 2 x [128 v][64 k]
+constexpr uint32_t UT = ST + 32768;                   // U~^T, then the O tile
+constexpr uint32_t MISC = UT + 16384;                 // barriers, TMEM address
+static_assert(MISC + 256 <= kSmemBytes && (2 * kProdBytes) % 1024 == 0, "light shared memory plan");
+}  // namespace light
+
+template <typename OutT>
+__device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const CUtensorMap& tm_o, const ChunkArgs& p,
+                                                 const SegItem it) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw;
+    const uint32_t sbase = smem_u32(sm);
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) report_timeout(15);
+        return;
+    }
+    constexpr bool kStageO = sizeof(OutT) == 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, part = warp >> 2;
+    const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + light::MISC);  // [0],[1]: buffer loads; [2]: MMA
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+    constexpr int kLoader = 96;
+
+    if (warp == 0) {
+        tmem_alloc(sTmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbar_init();
+    }
+    if (tid == 64) {
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_o);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *sTmem;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const int vrow = quad * 32 + lane;
+    const int t_begin = it.tok_begin, t_end = it.tok_end;
+    const int nchunks = (t_end - t_begin + kC - 1) / kC;
+    auto image = [&](int c) { return p.prod + ((size_t(item_id) * p.prodL + c) * H + h) * kProdBytes; };
+    auto issue = [&](int c) {  // chunk c's image and V into buffer c & 1
+        const int b = c & 1;
+        mbar_arrive_expect_tx(&bars[b], kProdBytes + 16384u);
+        bulk_load_1d(sm + light::PROD + b * kProdBytes, image(c), kProdBytes, &bars[b]);
+        tma_load_3d(sm + light::V + b * 16384, &tm_v, &bars[b], 0, h, t_begin + c * kC);
+        tma_load_3d(sm + light::V + b * 16384 + 8192, &tm_v, &bars[b], 64, h, t_begin + c * kC);
+    };
+    int pend[2] = {-1, -1};  // loader thread: the chunk whose load into buffer b is in flight
+    if (tid == kLoader) {
+        for (int c = 0; c < 2 && c < nchunks; ++c) {
+            issue(c);
+            pend[c] = c;
+        }
+    }
+    {  // start state into TMEM (S^T: lane = v, column = k)
+        const float* src = p.segS + (size_t(item_id) * H + h) * (kD * kD);
+#pragma unroll 1
+        for (int cb = 0; cb < 2; ++cb) {
+            float buf[16];
+            const int k0 = part * 32 + cb * 16;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) buf[j] = src[size_t(k0 + j) * kD + vrow];
+            tmem_st16(tbase + TM_S + lane_off + k0, buf);
+        }
+        tmem_wait_st();
+    }
+    const uint32_t id_u = idesc_bf16(128, 64, 1, 0);     // V^T (MN) x (T beta)^T (K)
+    const uint32_t id_so2 = idesc_bf16(128, 128, 0, 1);  // S'^T (K) x [-W^T | Qp] (MN)
+    const uint32_t id_os = idesc_bf16(128, 192, 0, 0);   // U~^T (K) x [P^T | Km] (K)
+    uint32_t ph_mma = 0;
+    bool aborted = false;
+
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c & 1, t0 = t_begin + c * kC, len = min(kC, t_end - t0);
+        uint8_t* img = sm + light::PROD + b * kProdBytes;
+        const uint32_t simg = sbase + light::PROD + b * kProdBytes;
+        bool ok = mbar_wait(&bars[b], uint32_t((c >> 1) & 1), 1);
+        if (tid == kLoader) pend[b] = -1;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        {  // S <- S post(prev); bf16 S' = S e^{mp}; TMEM S = S e^{mk}; O^T = 0
+            const float* frOp = reinterpret_cast<const float*>(img + PI_FR);
+            const float* frAcc = frOp + 128;
+            float x[32];
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) tmem_ld16(tbase + TM_S + lane_off + part * 32 + cb * 16, x + cb * 16);
+            tmem_wait_ld();
+            const uint32_t dst = sbase + light::ST + ((part >> 1) ? 16384u : 0u);
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                const int k0 = part * 32 + cb * 16, ck = (part & 1) * 4 + cb * 2;
+                uint32_t pk[8];
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 fo = *reinterpret_cast<const float4*>(frOp + k0 + j);
+                    const float4 fa = *reinterpret_cast<const float4*>(frAcc + k0 + j);
+                    float* xx = x + cb * 16 + j;
+                    pk[j >> 1] = pack_bf16x2(xx[0] * fo.x, xx[1] * fo.y);
+                    pk[(j >> 1) + 1] = pack_bf16x2(xx[2] * fo.z, xx[3] * fo.w);
+                    xx[0] *= fa.x;
+                    xx[1] *= fa.y;
+                    xx[2] *= fa.z;
+                    xx[3] *= fa.w;
+                }
+                st_shared_v4(dst + sw128_chunk(vrow, ck), pk[0], pk[1], pk[2], pk[3]);
+                st_shared_v4(dst + sw128_chunk(vrow, ck + 1), pk[4], pk[5], pk[6], pk[7]);
+            }
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) tmem_st16(tbase + TM_S + lane_off + part * 32 + cb * 16, x + cb * 16);
+            float z[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) z[j] = 0.f;
+            tmem_st16(tbase + TM_O + lane_off + part * 16, z);
+            tmem_wait_st();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {  // U^T = V^T (T beta)^T, then [U~ | O] += S'^T [-W^T | Qp]
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_bf16(tbase + TM_U, sdesc_sw128(sbase + light::V + b * 16384 + ks * 2048, 8192, 1024),
+                          sdesc_sw128(simg + PI_TB + ks * 32, 16, 1024), id_u, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_bf16(tbase + TM_U, sdesc_sw128(sbase + light::ST + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                          sdesc_sw128(simg + PI_WN + ks * 2048, PI_QP - PI_WN, 1024), id_so2, 1);
+            umma_commit(&bars[2]);
+        }
+        ok = mbar_wait(&bars[2], ph_mma, 5);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (tid == 0) bulk_wait_read0();  // the previous O tile (over U~^T) is read out
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        {  // U~^T -> smem
+            float u[16];
+            tmem_ld16(tbase + TM_U + lane_off + part * 16, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 2; ++q4)
+                st_shared_v4(sbase + light::UT + sw128_chunk(vrow, part * 2 + q4), pack_bf16x2(u[q4 * 8 + 0], u[q4 * 8 + 1]),
+                             pack_bf16x2(u[q4 * 8 + 2], u[q4 * 8 + 3]), pack_bf16x2(u[q4 * 8 + 4], u[q4 * 8 + 5]),
+                             pack_bf16x2(u[q4 * 8 + 6], u[q4 * 8 + 7]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {  // [O | S] += U~^T [P^T | Km]
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_bf16(tbase + TM_O, sdesc_sw128(sbase + light::UT + ks * 32, 16, 1024),
+                          sdesc_sw128(simg + PI_P + ks * 32, 16, 1024), id_os, 1);
+            umma_commit(&bars[2]);
+        }
+        ok = mbar_wait(&bars[2], ph_mma, 6);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        if (tid == kLoader && c + 2 < nchunks) {  // buffer b is consumed: chunk c+2 goes there
+            issue(c + 2);
+            pend[b] = c + 2;
+        }
+        bool staged = false;
+        {  // O^T -> o[t0 + r, h, v]
+            float ov[16];
+            tmem_ld16(tbase + TM_O + lane_off + part * 16, ov);
+            tmem_wait_ld();
+            if (kStageO && len == kC) {
+                uint8_t* so = sm + light::UT + (vrow >> 6) * 8192;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    *reinterpret_cast<__nv_bfloat16*>(so + sw128_off(part * 16 + j, vrow & 63)) =
+                        __float2bfloat16_rn(ov[j]);
+                fence_async_smem();
+                staged = true;
+            } else {
+                OutT* o = static_cast<OutT*>(p.o);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int r = part * 16 + j;
+                    if (r < len) o[(size_t(t0 + r) * H + h) * kD + vrow] = from_f32<OutT>(ov[j]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (staged && tid == 0) {
+            tma_store_3d(&tm_o, sm + light::UT, 0, h, t0);
+            tma_store_3d(&tm_o, sm + light::UT + 8192, 64, h, t0);
+            bulk_commit();
+        }
+    }
+    if (aborted) {  // let copies and MMAs still in flight land before shared memory and TMEM are released
+        if (tid == kLoader) {
+            for (int b = 0; b < 2; ++b)
+                if (pend[b] >= 0) mbar_wait(&bars[b], uint32_t((pend[b] >> 1) & 1), 7);
+        }
+        if (tid == 0) mbar_wait(&bars[2], ph_mma, 7);
+    }
+    if (tid == 0) bulk_wait0();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
 // Phase 1 (and the only launch of an unsegmented call): segment 0's output, and
@@ -1093,7 +1392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
 }
 
-// Phase 2: the outputs of segments 1..G-1 from the combine pass's start states.
+// Phase 2: the outputs of segments 1..G-1 from the combine pass's start states;
+// the middle segments reuse the products their map pass exported.
 template <typename OutT, bool kScalarGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1101,14 +1401,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
     if (int(blockIdx.x) >= *p.n_items) return;
     const SegItem it = p.items[blockIdx.x];
-    if (it.g >= 1) chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+    if (it.g >= 1 && it.g < it.G - 1 && p.prod)  // its map pass exported the chunk products
+        chunk_light_body<OutT>(tm_v, tm_o, p, it);
+    else if (it.g >= 1)
+        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
 }
 
 // ---------------------------------------------------------------- plan
 // One CTA: per sequence n, G_n = max(1, ceil(chunks_n / L)) segments; writes the
 // segment table in sequence order and the item count.
+// Segment 0 of a sequence has L0 chunks, the others L (the last one the rest).
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, int T, int L, SegItem* items,
-                                                    int* n_items, int max_items) {
+                                                    int* n_items, int max_items, int L0) {
     using Scan = cub::BlockScan<int, 1024>;
     __shared__ typename Scan::TempStorage tmp;
     __shared__ int s_base;
@@ -1120,8 +1424,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
         if (n < N) {
             sb = cu ? cu[n] : n * T;
             se = cu ? cu[n + 1] : (n + 1) * T;
-            const int nch = (se - sb + kC - 1) / kC;
-            G = nch > 0 ? (nch + L - 1) / L : 1;
+            const long long nch = (se - sb + kC - 1) / kC;
+            G = nch > L0 ? 1 + int((nch - L0 + L - 1) / L) : 1;
         }
         int off = 0, tot = 0;
         Scan(tmp).ExclusiveSum(G, off, tot);
@@ -1132,8 +1436,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
                 if (id >= max_items) break;
                 SegItem s;
                 s.seq = n;
-                s.tok_begin = int(min((long long)se, sb + (long long)g * L * kC));
-                s.tok_end = int(min((long long)se, sb + (long long)(g + 1) * L * kC));
+                const long long c0 = g == 0 ? 0 : L0 + (long long)(g - 1) * L;
+                const long long c1 = g == 0 ? L0 : c0 + L;
+                s.tok_begin = int(min((long long)se, sb + c0 * kC));
+                s.tok_end = int(min((long long)se, sb + c1 * kC));
                 s.g = g;
                 s.G = G;
                 s.first = off;
@@ -1157,12 +1463,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
 constexpr int kCombCols = 16;
 constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 64;
 
-__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
 
 __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const float* init,
                                                       const float* segN, const float* segXt, float* segS, int H) {
@@ -1296,6 +1596,8 @@ int device_sm_count() {
 }
 
 struct ChunkPlan {
+    size_t off_prod, prod_bytes, total_min;  // product images; workspace without them
+    int L0;                                  // chunks of segment 0 (L for the others)
     int N, L, max_items;
     long long Ttot;
     bool scan;
@@ -1310,15 +1612,23 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     pl.Ttot = varlen ? (long long)T : (long long)B * T;
     const long long chunks_bound = (pl.Ttot + kC - 1) / kC + pl.N;
     const long long pairs = (long long)pl.N * H;
-    int L = 1 << 30;
+    int L = 1 << 30, L0 = 1 << 30;
     if (pairs > 0 && pairs * 3 <= nsm) {
-        const long long G = nsm / pairs + 1;  // segments per sequence: G-1 CTAs per pair in each phase
+        // segments per sequence: G-1 CTAs per pair in each phase.  The last segment is
+        // about kLastShare of the others: in phase 2 it runs the full kernel while the
+        // middle segments reuse their exported products (about that much cheaper).
+        // Segment 0 runs beside the maps in phase 1; kFirstShare sets its length relative
+        // to theirs (measured at B=1 H=16 T=65536: 0.85 and 1.0 tie, 1.15 is slower).
+        const long long Gm1 = nsm / pairs;
         const long long per_seq = (chunks_bound + pl.N - 1) / pl.N;
-        L = int((per_seq + G - 1) / G);
+        constexpr double kLastShare = 0.35, kFirstShare = 1.0;
+        L = int(std::ceil(double(per_seq) / (double(Gm1) - 1.0 + kFirstShare + kLastShare)));
         if (L < 1) L = 1;
-        if (per_seq < 3 * (long long)L) L = 1 << 30;  // too short to pay for the summary pass
+        L0 = std::max(L, int(std::lround(kFirstShare * L)));
+        if (per_seq < 3 * (long long)L) L = L0 = 1 << 30;  // too short to pay for the map pass
     }
     pl.L = L;
+    pl.L0 = L0;
     pl.scan = L < (1 << 30);
     pl.max_items = int(pl.N + (pl.scan ? (chunks_bound + L - 1) / L : 0));
     size_t off = 0;
@@ -1333,6 +1643,9 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     pl.off_q = off; off = up256(off + (need_qk ? tok : 0));
     pl.off_k = off; off = up256(off + (need_qk ? tok : 0));
     pl.off_v = off; off = up256(off + (dtype == KDA_FP32 ? tok : 0));
+    pl.total_min = off;
+    pl.prod_bytes = pl.scan ? size_t(pl.max_items) * size_t(L) * H * kProdBytes : 0;
+    pl.off_prod = off; off = up256(off + pl.prod_bytes);
     pl.total = off;
     return pl;
 }
@@ -1367,7 +1680,10 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
                      const char** why, int scalar_gate) {
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
-    if (ws_bytes < pl.total || (pl.total > 0 && ws == nullptr)) {
+    // A workspace of kda_chunk_fwd_workspace() bytes holds the exported chunk products of
+    // segmented calls; one of only total_min bytes runs the same schedule recomputing them.
+    const bool products = pl.scan && ws_bytes >= pl.total;
+    if (ws_bytes < pl.total_min || (pl.total_min > 0 && ws == nullptr)) {
         *why = "workspace smaller than kda_chunk_fwd_workspace()";
         return KDA_ERR_WORKSPACE;
     }
@@ -1420,11 +1736,13 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
 
     cudaEvent_t* ev = g_trace_events;
     if (ev) cudaEventRecord(ev[0], stream);
-    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items);
+    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0);
     if (ev) cudaEventRecord(ev[1], stream);
 
     ChunkArgs a{};
     a.beta = beta;
+    a.prod = products ? w + pl.off_prod : nullptr;
+    a.prodL = pl.L;
     a.gs = scalar_gate ? g : nullptr;
     a.init_state = init;
     a.final_state = fin;
@@ -1488,11 +1806,17 @@ extern "C" int kda_debug_warp_cycles(unsigned long long* out, int reset) {
 
 int chunk_segment_tokens(int B, int T, int H, int num_seqs) {
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count());
-    return pl.scan ? pl.L * kC : 0;
+    return pl.scan ? pl.L0 * kC : 0;
 }
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
     return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total;
+}
+
+// The smallest workspace kda_chunk_fwd accepts (the segmented schedule then recomputes
+// the chunk products in its output pass instead of reading them back).
+size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
+    return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total_min;
 }
 
 }  // namespace kda

@@ -34,6 +34,7 @@ constexpr int kNoAllocMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
+size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 
 // Device address of g_noalloc_scratch on the current device (looked up once).
 static void* noalloc_scratch(const char** why) {
@@ -72,7 +73,10 @@ extern "C" int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v
     if (B < 0 || T < 0 || H < 0 || num_seqs < 0)
         return kda_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H, dtype,
                              scale, l2norm_qk, nullptr, 0, stream);  // reports the bad size
-    const size_t need = chunk_workspace_bytes(B, T, H, cu_seqlens ? num_seqs : 0, dtype, l2norm_qk);
+    // the full workspace if it fits (the fastest schedule), else the smallest accepted one
+    const int ns = cu_seqlens ? num_seqs : 0;
+    size_t need = chunk_workspace_bytes(B, T, H, ns, dtype, l2norm_qk);
+    if (need > kNoAllocScratchBytes) need = chunk_workspace_bytes_min(B, T, H, ns, dtype, l2norm_qk);
     if (need > kNoAllocScratchBytes) {
         snprintf(t_last_error, sizeof(t_last_error),
                  "kda_chunk_fwd_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte static "

@@ -113,24 +113,34 @@ int kda_set_trace_events(void *events, int n_events);
  *                  must be 1 and N = num_seqs >= 1.  Empty sequences are allowed.
  *                  The offsets are read on the device only (never copied back).
  *   scale     multiplies q (1.0 = o_t = S_t^T q_t).
- *   workspace      device scratch of at least kda_chunk_fwd_workspace(...)
- *                  bytes, 256-byte aligned; contents need not be initialised
- *                  and are clobbered.
+ *   workspace      device scratch of at least kda_chunk_fwd_workspace_min(...)
+ *                  bytes (kda_chunk_fwd_workspace(...) for the fastest
+ *                  schedule), 256-byte aligned; contents need not be
+ *                  initialised and are clobbered.
  *
  * Tensor cores compute the chunk contractions with bf16 operands and fp32
  * accumulation; the state is carried in fp32.  fp32 inputs are rounded to
  * bf16 where they feed the tensor cores.
  */
 /* How a kda_chunk_fwd call with these sizes on the current device is split:
- * 0 when every (sequence, head) runs in one CTA; otherwise the segment length
- * in tokens.  A segmented call runs its first segment and the segment maps in
- * one launch, then the combine pass, then the outputs of the later segments.
- * Informational (profiling); the result never changes what is computed. */
+ * 0 when every (sequence, head) runs in one CTA; otherwise the length in tokens
+ * of each sequence's first segment.  A segmented call runs the first segments'
+ * outputs and the later segments' maps in one launch, then the combine pass,
+ * then the later segments' outputs.  Informational (profiling); it never
+ * changes what is computed. */
 int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs);
 
 /* Workspace bytes for a kda_chunk_fwd call with the same B, T, H, num_seqs
  * (0 = dense), dtype and l2norm_qk, on the current device. */
 size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk);
+
+/* The smallest workspace kda_chunk_fwd accepts for the same arguments.  With a
+ * workspace of at least kda_chunk_fwd_workspace() bytes a segmented call keeps
+ * each segment map pass's per-chunk products (about 66 KB per chunk and head,
+ * e.g. ~1.2 GB at B=1 H=16 T=65536) and its output pass reads them back instead
+ * of recomputing them; with less (but at least this many) bytes it recomputes
+ * them.  Both give bit-identical results; the first is faster. */
+size_t kda_chunk_fwd_workspace_min(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk);
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
                   const float *initial_state, float *final_state, void *o, const int32_t *cu_seqlens,

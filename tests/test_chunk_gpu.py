@@ -134,3 +134,27 @@ def test_prefill_64k_sampled_heads(kda):
     inp = synth.op_inputs(**synth.prefill_sweep(65536), device="cuda")
     eo, es = run_both(kda, inp, heads=[0, 11])
     assert eo < TOL and es < TOL, (eo, es)
+
+
+@pytest.mark.parametrize("scalar_gate", [False, True])
+def test_both_segmented_schedules_give_identical_bits(kda, scalar_gate):
+    """With the full workspace the output pass of middle segments reads back the
+    chunk products their map pass exported; with the minimal one it recomputes
+    them.  The same values go through the same MMAs either way."""
+    B, T, H = 1, 3000, 16
+    inp = synth.op_inputs(B=B, H=H, T=T, s0_std=0.02, seed=16, scalar_gate=scalar_gate)
+    d = {n: inp[n].cuda() for n in ("q", "k", "v", "g", "beta")}
+    if scalar_gate:
+        d["g"] = d["g"][..., 0].contiguous()
+    fn = kda.gdn_chunk_fwd if scalar_gate else kda.chunk_fwd
+    lib = kda.lib()
+    full = lib.kda_chunk_fwd_workspace(B, T, H, 0, 0, 0)
+    small = lib.kda_chunk_fwd_workspace_min(B, T, H, 0, 0, 0)
+    assert lib.kda_chunk_fwd_segment_tokens(B, T, H, 0) > 0 and small < full
+    res = []
+    for nbytes in (full, small):
+        ws = torch.empty(nbytes, device="cuda", dtype=torch.uint8)
+        res.append(fn(*(d[n] for n in ("q", "k", "v", "g", "beta")), initial_state=inp["s0"].cuda(), workspace=ws))
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
