@@ -59,7 +59,7 @@ def _load():
     lib.kda_chunk_fwd_workspace.restype = sz
     lib.kda_chunk_fwd_workspace_min.argtypes = [i, i, i, i, i, i]
     lib.kda_chunk_fwd_workspace_min.restype = sz
-    lib.kda_chunk_fwd_segment_tokens.argtypes = [i, i, i, i]
+    lib.kda_chunk_fwd_segment_tokens.argtypes = [i, i, i, i, ctypes.POINTER(ctypes.c_int)]
     lib.kda_chunk_fwd_segment_tokens.restype = i
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i
@@ -141,6 +141,13 @@ def set_trace_events(events):
 
 
 _trace_keep = None
+
+
+def chunk_fwd_segments(B, T, H, num_seqs=0):
+    """(first segment tokens, following segment tokens) of a kda_chunk_fwd call; (0, 0) if unsegmented."""
+    mid = ctypes.c_int(0)
+    first = int(_lib.kda_chunk_fwd_segment_tokens(B, T, H, num_seqs, ctypes.byref(mid)))
+    return first, mid.value
 
 
 def chunk_fwd_workspace_bytes(B, T, H, num_seqs=0, dtype=KDA_BF16, l2norm_qk=False) -> int:

@@ -17,7 +17,7 @@ int launch_recurrent_bwd(const void* q, const void* k, const void* v, const floa
                          const float* init, const void* dout, const float* dfinal, float* dq, float* dk, float* dv,
                          float* dg, float* dbeta, float* dinit, int B, int Tn, int H, int dtype, float scale,
                          void* ws, size_t ws_bytes, cudaStream_t stream, const char** why);
-int chunk_segment_tokens(int B, int T, int H, int num_seqs);
+int chunk_segment_tokens(int B, int T, int H, int num_seqs, int* middle);
 size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
@@ -91,9 +91,10 @@ int kda_device_status(void* stream) {
     return KDA_OK;
 }
 
-int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs) {
+int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int* middle_tokens) {
+    if (middle_tokens) *middle_tokens = 0;
     if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;
-    return chunk_segment_tokens(B, T, H, num_seqs);
+    return chunk_segment_tokens(B, T, H, num_seqs, middle_tokens);
 }
 
 size_t kda_chunk_fwd_workspace_min(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk) {

@@ -1804,8 +1804,9 @@ extern "C" int kda_debug_warp_cycles(unsigned long long* out, int reset) {
 }
 #endif
 
-int chunk_segment_tokens(int B, int T, int H, int num_seqs) {
+int chunk_segment_tokens(int B, int T, int H, int num_seqs, int* middle) {
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count());
+    if (middle) *middle = pl.scan ? pl.L * kC : 0;
     return pl.scan ? pl.L0 * kC : 0;
 }
 

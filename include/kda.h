@@ -124,11 +124,12 @@ int kda_set_trace_events(void *events, int n_events);
  */
 /* How a kda_chunk_fwd call with these sizes on the current device is split:
  * 0 when every (sequence, head) runs in one CTA; otherwise the length in tokens
- * of each sequence's first segment.  A segmented call runs the first segments'
- * outputs and the later segments' maps in one launch, then the combine pass,
- * then the later segments' outputs.  Informational (profiling); it never
- * changes what is computed. */
-int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs);
+ * of each sequence's first segment, with the length of the following segments
+ * (the last one holds the rest) in *middle_tokens when that is not NULL.  A
+ * segmented call runs the first segments' outputs and the later segments' maps
+ * in one launch, then the combine pass, then the later segments' outputs.
+ * Informational (profiling); it never changes what is computed. */
+int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int *middle_tokens);
 
 /* Workspace bytes for a kda_chunk_fwd call with the same B, T, H, num_seqs
  * (0 = dense), dtype and l2norm_qk, on the current device. */
