@@ -276,22 +276,15 @@ def run_ours(args):
     assert kda.device_status() == 0
     value = world * T / (ms / 1e3)
 
-    # Roofline per launch, algorithmic bytes of the tokens each processes: phase 1 writes the
-    # outputs of each sequence's first segment (q, k, v, g, beta read, o written: 1540 B per
-    # token-head) and reads the inputs of the map segments (1284 B, no output); phase 2 writes
-    # the outputs of all later segments (1540 B).  The longer launch is reported as dominant.
+    # Roofline per launch, algorithmic bytes of the tokens each processes: phase 1 runs every
+    # segment's map (q, k, v, g, beta read, no output: 1284 B per token-head); phase 2 writes
+    # every token's output (1540 B).  Unsegmented calls run one launch, timed as phase 2.  The
+    # longer launch is reported as dominant.
     seg0, mid = kda.chunk_fwd_segments(1, T, H_PREFILL)
-    if seg0 == 0:  # unsegmented: one launch, timed as phase 2
-        p1_bytes, p2_bytes = 0, BYTES_PER_TOKEN_HEAD * T * H_PREFILL
-        map_tokens = 0
-    else:
-        rest = T - min(seg0, T)
-        n_later = (rest + mid - 1) // mid  # segments after the first; the last holds the remainder
-        map_tokens = max(0, n_later - 1) * mid
-        p1_bytes = (BYTES_PER_TOKEN_HEAD * min(seg0, T) + (BYTES_PER_TOKEN_HEAD - 2 * D) * map_tokens) * H_PREFILL
-        p2_bytes = BYTES_PER_TOKEN_HEAD * rest * H_PREFILL
-    launches = {"phase1_first_segments_and_maps": {"ms": sum_ms, "algorithmic_bytes": p1_bytes},
-                "phase2_later_segments": {"ms": out_ms, "algorithmic_bytes": p2_bytes}}
+    p1_bytes = 0 if seg0 == 0 else (BYTES_PER_TOKEN_HEAD - 2 * D) * T * H_PREFILL
+    p2_bytes = BYTES_PER_TOKEN_HEAD * T * H_PREFILL
+    launches = {"phase1_segment_maps": {"ms": sum_ms, "algorithmic_bytes": p1_bytes},
+                "phase2_segment_outputs": {"ms": out_ms, "algorithmic_bytes": p2_bytes}}
     for rec in launches.values():
         rec["achieved_gbs"] = rec["algorithmic_bytes"] / (rec["ms"] / 1e3) / 1e9 if rec["ms"] > 0 else 0.0
         rec["frac"] = rec["achieved_gbs"] / hbm_peak
@@ -304,8 +297,8 @@ def run_ours(args):
                 "kernel": dom, "launches": launches, "segment_tokens": {"first": seg0, "following": mid},
                 "peak_kind": peak_kind,
                 "step_frac": BYTES_PER_TOKEN_HEAD * T * H_PREFILL / (ms / 1e3) / 1e9 / hbm_peak,
-                "kernel_ms": {"plan": plan_ms, "first_segment_and_maps": sum_ms, "combine": comb_ms,
-                              "later_segments": out_ms},
+                "kernel_ms": {"plan": plan_ms, "segment_maps": sum_ms, "combine": comb_ms,
+                              "segment_outputs": out_ms},
                 "tensor_tflops_step": FLOP_PER_TOKEN_HEAD * T * H_PREFILL / (ms / 1e3) / 1e12,
                 "tensor_peak": tc_peak}
 
@@ -375,12 +368,17 @@ def run_ours(args):
         gstep()
     barrier()
     torch.cuda.synchronize()
+    gtr = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        kda.set_trace_events(gtr[i])
         gstep()
     end.record(stream)
+    kda.set_trace_events(None)
     torch.cuda.synchronize()
     gdn_ms = max_over_ranks(start.elapsed_time(end) / args.steps)
+    gdn_kernel_ms = {name: statistics.mean(tr[a].elapsed_time(tr[a + 1]) for tr in gtr)
+                     for a, name in enumerate(("plan", "segment_maps", "combine", "segment_outputs"))}
     assert kda.device_status() == 0
     gdn_bytes = GDN_BYTES_PER_TOKEN_HEAD * T * H_PREFILL
 
@@ -477,7 +475,7 @@ def run_ours(args):
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,
-                    "step_frac": gdn_bytes / (gdn_ms / 1e3) / 1e9 / hbm_peak},
+                    "step_frac": gdn_bytes / (gdn_ms / 1e3) / 1e9 / hbm_peak, "kernel_ms": gdn_kernel_ms},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

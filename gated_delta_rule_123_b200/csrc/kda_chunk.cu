@@ -203,10 +203,11 @@ constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output from the segment's true start state (the initial state
 //                   for segment 0, the combine pass's result for the others).
-// A segmented sequence runs in two phases of launches: phase 1 computes the
-// output of segment 0 (whose start state is known) side by side with the maps of
-// segments 1..G-2; after the combine pass, phase 2 computes the outputs of
-// segments 1..G-1.  Both phases keep G-1 CTAs per (sequence, head) busy.
+// A segmented sequence runs in two phases of launches: phase 1 computes the maps
+// of its G equal segments (exporting each chunk's products when the workspace has
+// room); after the combine pass has chained the maps from the initial state,
+// phase 2 computes every segment's output.  Both keep G CTAs per (sequence, head)
+// busy (G-1 in phase 1 without the export: the last segment needs no map).
 // kScalarGate = true: one log-gate per (token, head) (gated DeltaNet); every key
 // channel shares it, so the decay factors are per row instead of per element.
 constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
@@ -1104,8 +1105,6 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
         } else if (it.g == it.G - 1) {
             if (p.final_state) dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
-        } else if (it.g == 0) {  // segment 1's start state, for the combine pass and phase 2
-            dstS = p.segS + (size_t(item_id + 1) * H + h) * (kD * kD);
         }
         tc_fence_after();
         auto store = [&](uint32_t tcol, float* dst) {
@@ -1158,8 +1157,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 // chunk it loads the product image (double-buffered, one bulk copy) and V, and
 // runs only the state chain -- the frame pass, U^T = V^T (T beta)^T followed by
 // [U~ | O] += S'^T [-W^T | Qp] in one MMA group, the U~ spill, [O | S] +=
-// U~^T [P | Km], and the O store.  The segment's end state is not needed (the
-// combine pass produced the next segment's start state).
+// U~^T [P | Km], and the O store.  Only the last segment's end state is stored
+// (the combine pass produced the other segments' successors' start states).
 namespace light {
 constexpr uint32_t PROD = 0;                          // 2 product images
 constexpr uint32_t V = 2 * kProdBytes;                // 2 x [64 tok][128 v]
@@ -1224,14 +1223,15 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
             pend[c] = c;
         }
     }
-    {  // start state into TMEM (S^T: lane = v, column = k)
-        const float* src = p.segS + (size_t(item_id) * H + h) * (kD * kD);
+    {  // start state into TMEM (S^T: lane = v, column = k): the initial state (or zero) for segment 0
+        const float* src = it.g > 0 ? p.segS + (size_t(item_id) * H + h) * (kD * kD)
+                                    : (p.init_state ? p.init_state + (size_t(it.seq) * H + h) * (kD * kD) : nullptr);
 #pragma unroll 1
         for (int cb = 0; cb < 2; ++cb) {
             float buf[16];
             const int k0 = part * 32 + cb * 16;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) buf[j] = src[size_t(k0 + j) * kD + vrow];
+            for (int j = 0; j < 16; ++j) buf[j] = src ? src[size_t(k0 + j) * kD + vrow] : 0.f;
             tmem_st16(tbase + TM_S + lane_off + k0, buf);
         }
         tmem_wait_st();
@@ -1370,6 +1370,19 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
                 if (pend[b] >= 0) mbar_wait(&bars[b], uint32_t((pend[b] >> 1) & 1), 7);
         }
         if (tid == 0) mbar_wait(&bars[2], ph_mma, 7);
+    } else if (it.g == it.G - 1 && p.final_state && nchunks > 0) {
+        // end state = S^T(TMEM) x post(last chunk); the last image (never reloaded) holds post
+        const float* post = reinterpret_cast<const float*>(sm + light::PROD + ((nchunks - 1) & 1) * kProdBytes + PI_FR) + 256;
+        float* dst = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
+#pragma unroll 1
+        for (int cb = 0; cb < 2; ++cb) {
+            const int k0 = part * 32 + cb * 16;
+            float x[16];
+            tmem_ld16(tbase + TM_S + lane_off + k0, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) dst[size_t(k0 + j) * kD + vrow] = x[j] * post[k0 + j];
+        }
     }
     if (tid == 0) bulk_wait0();
     tc_fence_before();
@@ -1377,8 +1390,10 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
     if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
-// Phase 1 (and the only launch of an unsegmented call): segment 0's output, and
-// the maps of segments 1..G-2.
+// Phase 1 (and the only launch of an unsegmented call): the maps of every
+// segment of a segmented sequence (the last segment's map only exports its chunk
+// products, and runs only when there is room for them), and the whole output of
+// an unsegmented one.  Segmented calls thus run one code path on every SM.
 template <typename OutT, bool kScalarGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1386,14 +1401,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
     if (int(blockIdx.x) >= *p.n_items) return;
     const SegItem it = p.items[blockIdx.x];
-    if (it.g == 0)
+    if (it.G == 1)
         chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
-    else if (it.g < it.G - 1)
+    else if (it.g < it.G - 1 || p.prod)
         chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
 }
 
-// Phase 2: the outputs of segments 1..G-1 from the combine pass's start states;
-// the middle segments reuse the products their map pass exported.
+// Phase 2: the outputs of every segment of a segmented sequence from its start
+// state (the initial state, or the combine pass's), reusing the chunk products
+// the map pass exported when there was room for them.
 template <typename OutT, bool kScalarGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1401,9 +1417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
     if (int(blockIdx.x) >= *p.n_items) return;
     const SegItem it = p.items[blockIdx.x];
-    if (it.g >= 1 && it.g < it.G - 1 && p.prod)  // its map pass exported the chunk products
+    if (it.G == 1) return;  // its output was written in phase 1
+    if (p.prod)
         chunk_light_body<OutT>(tm_v, tm_o, p, it);
-    else if (it.g >= 1)
+    else
         chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
 }
 
@@ -1469,7 +1486,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
     const int item = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
     if (item >= *n_items) return;
     const SegItem it = items[item];
-    if (it.g != 0 || it.G < 3) return;  // S_1 comes from phase 1; S_2.. are chained here
+    if (it.g != 0 || it.G < 2) return;
     extern __shared__ __align__(128) uint8_t csm[];
     float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
     float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
@@ -1484,23 +1501,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
         fence_mbar_init();
     }
     __syncthreads();
-    // step j = 0, 1, ... maps S_{j+1} to S_{j+2} with segment j+1's map
+    // step j = 0, 1, ..., G-2 maps S_j to S_{j+1} with segment j's map (S_0 = the initial state)
     auto fetch = [&](int j) {
         mbar_arrive_expect_tx(&bar[j & 1], 65536u);
-        bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + 1 + j) * H * (kD * kD) + hs, 65536u, &bar[j & 1]);
+        bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + j) * H * (kD * kD) + hs, 65536u, &bar[j & 1]);
     };
     if (tid == 0) fetch(0);
-    (void)init;
     for (int e = tid; e < kD * kCombCols; e += 256) {
         const int kk = e / kCombCols, jj = e % kCombCols;
-        sS[e] = segS[size_t(item + 1) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj];
+        sS[e] = init ? init[size_t(it.seq) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] : 0.f;
     }
     __syncthreads();
     bool ok = true;
     int fetched = 1, j = 0;  // fetches issued (thread 0) and the step being consumed
-    for (; j + 2 < it.G; ++j) {
-        const int g = j + 1;  // the segment whose map this step applies
-        if (tid == 0 && j + 3 < it.G) {
+    for (; j + 1 < it.G; ++j) {
+        const int g = j;  // the segment whose map this step applies
+        if (tid == 0 && j + 2 < it.G) {
             fetch(j + 1);
             fetched = j + 2;
         }
@@ -1614,17 +1630,12 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     const long long pairs = (long long)pl.N * H;
     int L = 1 << 30, L0 = 1 << 30;
     if (pairs > 0 && pairs * 3 <= nsm) {
-        // segments per sequence: G-1 CTAs per pair in each phase.  The last segment is
-        // about kLastShare of the others: in phase 2 it runs the full kernel while the
-        // middle segments reuse their exported products (about that much cheaper).
-        // Segment 0 runs beside the maps in phase 1; kFirstShare sets its length relative
-        // to theirs (measured at B=1 H=16 T=65536: 0.85 and 1.0 tie, 1.15 is slower).
-        const long long Gm1 = nsm / pairs;
+        // G equal segments per sequence: one CTA per segment and pair in each phase
+        const long long G = nsm / pairs;
         const long long per_seq = (chunks_bound + pl.N - 1) / pl.N;
-        constexpr double kLastShare = 0.35, kFirstShare = 1.0;
-        L = int(std::ceil(double(per_seq) / (double(Gm1) - 1.0 + kFirstShare + kLastShare)));
+        L = int((per_seq + G - 1) / G);
         if (L < 1) L = 1;
-        L0 = std::max(L, int(std::lround(kFirstShare * L)));
+        L0 = L;
         if (per_seq < 3 * (long long)L) L = L0 = 1 << 30;  // too short to pay for the map pass
     }
     pl.L = L;

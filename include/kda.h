@@ -77,9 +77,9 @@ int kda_device_status(void *stream);
  * point to 5 cudaEvent_t created by the caller on the current device; every
  * later kda_chunk_fwd call on this thread records them on its stream around
  * its kernels: [0] before the plan kernel, [1] after it, [2] after the first
- * phase (segment 0's output and the later segments' maps; same as [1] when the
- * sequences are not segmented), [3] after the combine pass, [4] after the
- * outputs of the later segments (or of everything, unsegmented).  Pass NULL to
+ * phase (the segments' maps; same as [1] when the sequences are not
+ * segmented), [3] after the combine pass, [4] after the segments' outputs (or
+ * after the only launch, unsegmented).  Pass NULL to
  * stop.  The events stay owned by the caller. */
 int kda_set_trace_events(void *events, int n_events);
 
@@ -126,8 +126,8 @@ int kda_set_trace_events(void *events, int n_events);
  * 0 when every (sequence, head) runs in one CTA; otherwise the length in tokens
  * of each sequence's first segment, with the length of the following segments
  * (the last one holds the rest) in *middle_tokens when that is not NULL.  A
- * segmented call runs the first segments' outputs and the later segments' maps
- * in one launch, then the combine pass, then the later segments' outputs.
+ * segmented call runs the segments' maps in one launch, then the combine pass,
+ * then the segments' outputs in a second launch.
  * Informational (profiling); it never changes what is computed. */
 int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int *middle_tokens);
 
