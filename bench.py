@@ -254,20 +254,50 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert kda.device_status() == 0
 
-    # timed region: K steps, per-kernel trace events on the launching stream
+    def timed_steps(fn, traces):
+        """Time args.steps calls of fn with per-call trace events on the launching stream.
+        The calls are captured into one CUDA graph and replayed, so host-side jitter
+        between calls cannot leave the GPU idle; --eager times them as issued."""
+        for tr in traces:  # create the events outside the capture
+            for e in tr:
+                e.record(stream)
+        graph, timing = None, "eager: K calls issued back to back"
+        if not args.eager:
+            try:
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for i in range(args.steps):
+                        kda.set_trace_events(traces[i])
+                        fn()
+                kda.set_trace_events(None)
+                graph.replay()  # untimed: uploads the graph
+                torch.cuda.synchronize()
+                timing = "one CUDA graph of the K calls, replayed once"
+            except Exception as exc:  # fall back to timing the calls as issued
+                kda.set_trace_events(None)
+                graph = None
+                torch.cuda.synchronize()
+                print(f"bench: CUDA graph capture failed ({exc}); timing eagerly", file=sys.stderr)
+        assert kda.device_status() == 0
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                kda.set_trace_events(traces[i])
+                fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        kda.set_trace_events(None)
+        return start.elapsed_time(end) / args.steps, timing
+
+    # timed region: K steps
     traces = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(args.steps):
-        kda.set_trace_events(traces[i])
-        step()
-    end.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    kda.set_trace_events(None)
+    ms, timing = timed_steps(step, traces)
     clocks = sampler.stop()
-    ms = start.elapsed_time(end) / args.steps
     ms = max_over_ranks(ms)
     out_ms = statistics.mean(tr[3].elapsed_time(tr[4]) for tr in traces)
     sum_ms = statistics.mean(tr[1].elapsed_time(tr[2]) for tr in traces)
@@ -305,7 +335,7 @@ def run_ours(args):
     if args.prefill_only:
         if rank == 0:
             print(json.dumps({"metric": metric_name(), "value": value, "unit": "tokens/s", "ms_per_step": ms,
-                              "config": {"workload": f"KDA prefill B=1 H=16 T={T} (prefill only)"},
+                              "config": {"workload": f"KDA prefill B=1 H=16 T={T} (prefill only)", "timing": timing},
                               "roofline": roofline}), flush=True)
         if world > 1:
             dist.destroy_process_group()
@@ -369,14 +399,8 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     gtr = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    start.record(stream)
-    for i in range(args.steps):
-        kda.set_trace_events(gtr[i])
-        gstep()
-    end.record(stream)
-    kda.set_trace_events(None)
-    torch.cuda.synchronize()
-    gdn_ms = max_over_ranks(start.elapsed_time(end) / args.steps)
+    gdn_ms, _ = timed_steps(gstep, gtr)
+    gdn_ms = max_over_ranks(gdn_ms)
     gdn_kernel_ms = {name: statistics.mean(tr[a].elapsed_time(tr[a + 1]) for tr in gtr)
                      for a, name in enumerate(("plan", "segment_maps", "combine", "segment_outputs"))}
     assert kda.device_status() == 0
@@ -451,7 +475,8 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"KDA prefill B=1 H=16 T={T} d=128 bf16, fp32 g/beta/state "
                                    "(one independent sequence per GPU)",
-                       "l2": "inputs larger than L2 (1.6 GB per step)", "parallelism": f"replicas x{world}"},
+                       "l2": "inputs larger than L2 (1.6 GB per step)", "parallelism": f"replicas x{world}",
+                       "timing": timing},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -492,6 +517,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=T_PREFILL, help="prefill length (profiling runs use a smaller one)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and the CPU baseline")
+    ap.add_argument("--eager", action="store_true", help="time the prefill calls as issued, not as one CUDA graph")
     ap.add_argument("--layer-only", action="store_true", help="time only the KDA layer (profiling runs)")
     ap.add_argument("--warmup-seconds", type=float, default=1.5, help="minimum warm-up time (clock sampling)")
     args = ap.parse_args()

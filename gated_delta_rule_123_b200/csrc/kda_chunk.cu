@@ -108,7 +108,7 @@ static_assert(OFF_QP - OFF_KP == 32768 && OFF_QP - OFF_WN == 16384 && OFF_KM - O
 constexpr uint32_t MISC_BYTES = 7 * 1024;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES;
 static_assert(kSmemBytes <= 232448, "shared memory plan");
-// Summary pass reuses: S^T halves of X at OFF_Q / OFF_QP, U_X~^T at OFF_TB (16 KB).
+// The map pass keeps X' in TMEM (over [A;P]) and U_X~^T at OFF_TB (16 KB).
 
 // TMEM columns (512 allocated): U^T | O^T (or U_X^T) | S^T | [A;P] | W^T | X^T.
 // [U|O] and [O|S] are contiguous so one N=128 and one N=192 MMA can fill them.
@@ -645,9 +645,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             }
             tmem_wait_st();
         }
-        // the previous O tile (over U~^T / sA) and the previous chunk's exported -W^T (under T)
-        // have been read out
-        if (tid == 0 || (kSummary && tid == kExporter)) bulk_wait_read0();
+        // the previous O tile (over U~^T / sA) has been read out.  The exporter's groups are
+        // waited for after the U~/O MMA: that wait covers the previous chunk's -W^T (under T)
+        // before this chunk's solve, and this chunk's Qp / Km before they are rewritten.
+        if (tid == 0) bulk_wait_read0();
         if (fast) {
             ok = mbar_wait(&bars[2], ph_mma, 2);
             ph_mma ^= 1;
@@ -987,10 +988,11 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             if (!e_prep(c + 1)) { aborted = true; break; }
             __syncthreads();  // row-quarter sums (scalar gates: per-warp scans)
             e_head();
-            if (kScalarGate)
-                e_factors();  // the rows wait for the next barrier
-            else
-                e_rows(0, true);
+            if (kScalarGate) {
+                e_factors();
+                __syncthreads();  // every row's factors are in sFac
+            }
+            e_rows(0, true);
         }
         KDA_STAGE(16);
         ok = mbar_wait(&bars[2], ph_mma, 5);
@@ -1000,10 +1002,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         if (img && tid == kExporter) bulk_wait_read0();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(10);
-        if (has_next) {  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
-            if (kScalarGate) e_rows(0, true);
-            e_put_kq(0);
-        }
+        if (has_next) e_put_kq(0);  // Kp, Qp are free: the A/P, W and U~/O MMAs are done
         {  // U~^T (and U_X~^T) -> smem, lane = value channel, 16 tokens per thread
             auto spill = [&](uint32_t tcol, uint32_t dst_off) {
                 float u[16];
@@ -1520,16 +1519,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
             fetch(j + 1);
             fetched = j + 2;
         }
-        ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
-        if (__syncthreads_or(!ok)) break;
-        const float* X = sX + (j & 1) * kD * kD;
         const size_t base = size_t(item + g) * H * (kD * kD) + hs;
         float acc[2][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+        for (int r = 0; r < 2; ++r) {  // N_g's slice: requested before the wait for X_g
             const float4 n4 = *reinterpret_cast<const float4*>(segN + base + size_t(k0 + r) * kD + c0 + j0);
             acc[r][0] = n4.x; acc[r][1] = n4.y; acc[r][2] = n4.z; acc[r][3] = n4.w;
         }
+        ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
+        if (__syncthreads_or(!ok)) break;
+        const float* X = sX + (j & 1) * kD * kD;
 #pragma unroll 8
         for (int kp = 0; kp < kD; ++kp) {  // acc[k][j] += X[k][kp] S[kp][j] = Xt[kp][k] S[kp][j]
             const float2 xv = *reinterpret_cast<const float2*>(X + kp * kD + k0);
@@ -1686,6 +1685,17 @@ static int launch_phase_for(int dtype, int scalar_gate, dim3 grid, const CUtenso
                        : launch_phase<kPhase, __nv_bfloat16, false>(grid, mq, mk, mv, mg, mo, a, stream);
 }
 
+// Trace events are recorded as external event nodes when the stream is being
+// captured into a CUDA graph (so a replayed graph still times each launch), and
+// plainly otherwise (the external flag is refused outside a capture).
+static inline void trace_record(cudaEvent_t e, cudaStream_t stream) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, stream);
+}
+
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
@@ -1746,9 +1756,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     }
 
     cudaEvent_t* ev = g_trace_events;
-    if (ev) cudaEventRecord(ev[0], stream);
+    if (ev) trace_record(ev[0], stream);
     plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0);
-    if (ev) cudaEventRecord(ev[1], stream);
+    if (ev) trace_record(ev[1], stream);
 
     ChunkArgs a{};
     a.beta = beta;
@@ -1767,13 +1777,13 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     a.scale = scale;
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
     if (!pl.scan && ev) {  // one launch: it is timed as the output pass
-        cudaEventRecord(ev[2], stream);
-        cudaEventRecord(ev[3], stream);
+        trace_record(ev[2], stream);
+        trace_record(ev[3], stream);
     }
     const int r1 = launch_phase_for<1>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
     if (r1 != KDA_OK) return r1;
     if (pl.scan) {
-        if (ev) cudaEventRecord(ev[2], stream);
+        if (ev) trace_record(ev[2], stream);
         static bool comb_attr = false;
         if (!comb_attr) {
             if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombSmem) !=
@@ -1783,11 +1793,11 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         }
         combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
             items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
-        if (ev) cudaEventRecord(ev[3], stream);
+        if (ev) trace_record(ev[3], stream);
         const int r2 = launch_phase_for<2>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
         if (r2 != KDA_OK) return r2;
     }
-    if (ev) cudaEventRecord(ev[4], stream);
+    if (ev) trace_record(ev[4], stream);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         *why = cudaGetErrorString(e);

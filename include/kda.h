@@ -79,8 +79,10 @@ int kda_device_status(void *stream);
  * its kernels: [0] before the plan kernel, [1] after it, [2] after the first
  * phase (the segments' maps; same as [1] when the sequences are not
  * segmented), [3] after the combine pass, [4] after the segments' outputs (or
- * after the only launch, unsegmented).  Pass NULL to
- * stop.  The events stay owned by the caller. */
+ * after the only launch, unsegmented).  They are recorded with
+ * cudaEventRecordExternal, so a call captured into a CUDA graph records them
+ * as event nodes each time the graph runs.  Pass NULL to stop.  The events
+ * stay owned by the caller. */
 int kda_set_trace_events(void *events, int n_events);
 
 /* ------------------------------------------------------------------------

@@ -138,9 +138,9 @@ def test_prefill_64k_sampled_heads(kda):
 
 @pytest.mark.parametrize("scalar_gate", [False, True])
 def test_both_segmented_schedules_give_identical_bits(kda, scalar_gate):
-    """With the full workspace the output pass of middle segments reads back the
-    chunk products their map pass exported; with the minimal one it recomputes
-    them.  The same values go through the same MMAs either way."""
+    """With the full workspace each segment's output pass reads back the chunk
+    products its map pass exported; with the minimal one it recomputes them.  The
+    same values go through the same MMAs either way."""
     B, T, H = 1, 3000, 16
     inp = synth.op_inputs(B=B, H=H, T=T, s0_std=0.02, seed=16, scalar_gate=scalar_gate)
     d = {n: inp[n].cuda() for n in ("q", "k", "v", "g", "beta")}
@@ -158,3 +158,35 @@ def test_both_segmented_schedules_give_identical_bits(kda, scalar_gate):
     torch.cuda.synchronize()
     assert kda.device_status() == 0
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+
+
+def test_cuda_graph_replay_matches_eager_and_traces_launches(kda):
+    """A segmented call captured into a CUDA graph (as the benchmark times it) gives
+    the eager call's bits on replay, and trace events set during the capture time
+    each of its launches."""
+    B, T, H = 1, 3000, 16
+    inp = synth.op_inputs(B=B, H=H, T=T, s0_std=0.02, seed=17)
+    d = [inp[n].cuda() for n in ("q", "k", "v", "g", "beta")]
+    s0 = inp["s0"].cuda()
+    assert kda.chunk_fwd_segments(B, T, H)[0] > 0
+    ws = torch.empty(kda.chunk_fwd_workspace_bytes(B, T, H), device="cuda", dtype=torch.uint8)
+    o_ref, fs_ref = kda.chunk_fwd(*d, initial_state=s0, workspace=ws)
+    o, fs = torch.empty_like(o_ref), torch.empty_like(fs_ref)
+    torch.cuda.synchronize()
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for e in events:  # created outside the capture
+        e.record()
+    graph = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(graph):
+            kda.set_trace_events(events)
+            kda.chunk_fwd(*d, initial_state=s0, out=o, final_state=fs, workspace=ws)
+    finally:
+        kda.set_trace_events(None)
+    o.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    assert torch.equal(o, o_ref) and torch.equal(fs, fs_ref)
+    times = [events[i].elapsed_time(events[i + 1]) for i in range(4)]
+    assert all(t >= 0 for t in times) and times[1] > 0 and times[3] > 0, times
