@@ -1425,10 +1425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- plan
 // One CTA: per sequence n, G_n = max(1, ceil(chunks_n / L)) segments; writes the
-// segment table in sequence order and the item count.
+// segment table in sequence order, the item count and (if asked) each sequence's
+// first item.
 // Segment 0 of a sequence has L0 chunks, the others L (the last one the rest).
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, int T, int L, SegItem* items,
-                                                    int* n_items, int max_items, int L0) {
+                                                    int* n_items, int max_items, int L0, int* seq_first) {
     using Scan = cub::BlockScan<int, 1024>;
     __shared__ typename Scan::TempStorage tmp;
     __shared__ int s_base;
@@ -1446,6 +1447,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
         int off = 0, tot = 0;
         Scan(tmp).ExclusiveSum(G, off, tot);
         off += s_base;
+        if (seq_first && n < N) seq_first[n] = off;  // the item of its first segment
         if (n < N) {
             for (int g = 0; g < G; ++g) {
                 const int id = off + g;
@@ -1480,10 +1482,13 @@ constexpr int kCombCols = 16;
 constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 64;
 
 
-__global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const float* init,
-                                                      const float* segN, const float* segXt, float* segS, int H) {
-    const int item = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
-    if (item >= *n_items) return;
+__global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const int* seq_first,
+                                                      int N, const float* init, const float* segN,
+                                                      const float* segXt, float* segS, int H) {
+    const int n = blockIdx.x, h = blockIdx.y, z = blockIdx.z;  // one CTA per (sequence, head, slice)
+    if (n >= N) return;
+    const int item = seq_first[n];
+    if (item < 0 || item >= *n_items) return;
     const SegItem it = items[item];
     if (it.g != 0 || it.G < 2) return;
     extern __shared__ __align__(128) uint8_t csm[];
@@ -1616,7 +1621,7 @@ struct ChunkPlan {
     int N, L, max_items;
     long long Ttot;
     bool scan;
-    size_t off_items, off_count, off_segN, off_segX, off_segS, off_q, off_k, off_v, total;
+    size_t off_items, off_count, off_first, off_segN, off_segX, off_segS, off_q, off_k, off_v, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1644,6 +1649,7 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     size_t off = 0;
     pl.off_items = off; off = up256(off + sizeof(SegItem) * size_t(pl.max_items));
     pl.off_count = off; off = up256(off + 16);
+    pl.off_first = off; off = up256(off + (pl.scan ? sizeof(int) * size_t(pl.N) : 0));
     const size_t st = size_t(pl.max_items) * H * kD * kD * sizeof(float);
     pl.off_segN = off; off = up256(off + (pl.scan ? st : 0));
     pl.off_segX = off; off = up256(off + (pl.scan ? st : 0));
@@ -1757,7 +1763,8 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
 
     cudaEvent_t* ev = g_trace_events;
     if (ev) trace_record(ev[0], stream);
-    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0);
+    int* seq_first = pl.scan ? reinterpret_cast<int*>(w + pl.off_first) : nullptr;
+    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0, seq_first);
     if (ev) trace_record(ev[1], stream);
 
     ChunkArgs a{};
@@ -1791,8 +1798,8 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                 return KDA_ERR_CUDA;
             comb_attr = true;
         }
-        combine_kernel<<<dim3(unsigned(pl.max_items), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
-            items, n_items, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
+        combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
+            items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) trace_record(ev[3], stream);
         const int r2 = launch_phase_for<2>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
         if (r2 != KDA_OK) return r2;

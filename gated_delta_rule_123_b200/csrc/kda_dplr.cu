@@ -787,7 +787,7 @@ int launch_dplr_chunk_fwd(const void* q, const void* k, const void* v, const voi
         return KDA_ERR_CUDA;
     }
     // one segment per sequence
-    plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, 1 << 24, items, n_items, N, 1 << 24);
+    plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, 1 << 24, items, n_items, N, 1 << 24, nullptr);
     dplr::Args p{};
     p.beta = beta;
     p.init_state = init;
