@@ -1482,7 +1482,7 @@ constexpr int kCombCols = 16;
 constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 64;
 
 
-__global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, const int* n_items, const int* seq_first,
+__global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, const int* n_items, const int* seq_first,
                                                       int N, const float* init, const float* segN,
                                                       const float* segXt, float* segS, int H) {
     const int n = blockIdx.x, h = blockIdx.y, z = blockIdx.z;  // one CTA per (sequence, head, slice)
@@ -1534,12 +1534,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const SegItem* items, cons
         ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
         if (__syncthreads_or(!ok)) break;
         const float* X = sX + (j & 1) * kD * kD;
-#pragma unroll 8
-        for (int kp = 0; kp < kD; ++kp) {  // acc[k][j] += X[k][kp] S[kp][j] = Xt[kp][k] S[kp][j]
-            const float2 xv = *reinterpret_cast<const float2*>(X + kp * kD + k0);
-            const float4 sv = *reinterpret_cast<const float4*>(sS + kp * kCombCols + j0);
-            acc[0][0] += xv.x * sv.x; acc[0][1] += xv.x * sv.y; acc[0][2] += xv.x * sv.z; acc[0][3] += xv.x * sv.w;
-            acc[1][0] += xv.y * sv.x; acc[1][1] += xv.y * sv.y; acc[1][2] += xv.y * sv.z; acc[1][3] += xv.y * sv.w;
+#pragma unroll 1
+        for (int kb = 0; kb < kD; kb += 8) {  // acc[k][j] += X[k][kp] S[kp][j] = Xt[kp][k] S[kp][j]
+            float2 xv[8];  // 8 key steps' operands requested before their FMAs (hides the load latency)
+            float4 sv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                xv[u] = *reinterpret_cast<const float2*>(X + (kb + u) * kD + k0);
+                sv[u] = *reinterpret_cast<const float4*>(sS + (kb + u) * kCombCols + j0);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc[0][0] += xv[u].x * sv[u].x; acc[0][1] += xv[u].x * sv[u].y;
+                acc[0][2] += xv[u].x * sv[u].z; acc[0][3] += xv[u].x * sv[u].w;
+                acc[1][0] += xv[u].y * sv[u].x; acc[1][1] += xv[u].y * sv[u].y;
+                acc[1][2] += xv[u].y * sv[u].z; acc[1][3] += xv[u].y * sv[u].w;
+            }
         }
         __syncthreads();  // every thread has read sS and this X buffer
         const size_t out = size_t(item + g + 1) * H * (kD * kD) + hs;
