@@ -2,8 +2,8 @@
 """KDA on B200: prefill tokens/s at B=1, H=16, T=65536 and decode state GB/s.
 
 One step = one ``kda_chunk_fwd`` call over a B=1, H=16, T=65536, d=128 bf16
-sequence with a random fp32 initial state (plan; first segment's output with the
-later segments' maps; combine; the later segments' outputs).  The decode figure is measured in the same run on the
+sequence with a random fp32 initial state (plan; every segment's map with its
+chunk products exported; combine; every segment's output).  The decode figure is measured in the same run on the
 B=256, H=32 decode workload (512 MiB fp32 state updated in place).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
