@@ -127,6 +127,45 @@ def cpu_oracle_sample(T_s: int, H_s: int, seed: int = 77):
     return dt, oracle.num_threads()
 
 
+class Ranks:
+    """One process per GPU (or per CPU rank under gloo): rank ids from the launcher's
+    environment, a barrier, and the max of a per-rank number over all ranks.  Every rank
+    takes the same collective steps in the same order; the process group has a short
+    timeout so that ranks waiting for a missing peer end with an error."""
+
+    def __init__(self, backend: str, device=None, timeout_s: int = 120):
+        import datetime
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self._dist = dist
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self._dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        t = torch.tensor([x], device=self.device, dtype=torch.float64)
+        self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def seed(self, base: int) -> int:
+        """Each rank draws its own independent sequence (weak scaling)."""
+        return base + 1000 * self.rank
+
+    def close(self):
+        if self.world > 1:
+            self._dist.destroy_process_group()
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -179,35 +218,22 @@ def time_layer(kda, synth, dev, rank, time_calls, tc_peak, world):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
 
     import gated_delta_rule_123_b200 as kda
     import synth
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     T = args.T
     cfg = dict(synth.prefill_sweep(T))
-    cfg["seed"] += 1000 * rank
+    cfg["seed"] = ranks.seed(cfg["seed"])
     inp = synth.op_inputs(**cfg, device=dev)
     q, k, v, g, beta, s0 = (inp[n] for n in ("q", "k", "v", "g", "beta", "s0"))
     o = torch.empty_like(q)
@@ -238,8 +264,7 @@ def run_ours(args):
         if rank == 0:
             print(json.dumps({"metric": "KDA layer tokens/s", "value": layer["tokens_per_s"], "unit": "tokens/s",
                               "config": {"workload": layer["workload"]}, "layer": layer}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
+        ranks.close()
         return 0
 
     sampler = ClockSampler(local)
@@ -337,8 +362,7 @@ def run_ours(args):
             print(json.dumps({"metric": metric_name(), "value": value, "unit": "tokens/s", "ms_per_step": ms,
                               "config": {"workload": f"KDA prefill B=1 H=16 T={T} (prefill only)", "timing": timing},
                               "roofline": roofline}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
+        ranks.close()
         return 0
 
     # decode: B=256, H=32, state updated in place (inputs cycled from a pool of 8 seeded steps)
@@ -503,8 +527,7 @@ def run_ours(args):
                     "step_frac": gdn_bytes / (gdn_ms / 1e3) / 1e9 / hbm_peak, "kernel_ms": gdn_kernel_ms},
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
