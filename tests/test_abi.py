@@ -46,6 +46,32 @@ def test_workspace_queries(kda):
     assert kda.layer_fwd_workspace_bytes(65536, 2048, 16, 128, 8) > 65536 * 6416 * 2
 
 
+def test_segment_plan_on_148_sms(kda):
+    """Host-side plan (no device here: the library assumes a B200's 148 SMs).  With
+    P = sequences x heads <= 148/3 pairs, each sequence is cut into G = 148 // P equal
+    segments of L = ceil((chunks + 1) / G) chunks (the last holds the rest): one CTA per
+    segment and pair in each phase.  With more pairs every (sequence, head) runs whole."""
+    # B=1 H=16 T=65536: 1024 chunks, G = 9, L = ceil(1025 / 9) = 114 chunks
+    assert kda.chunk_fwd_segments(1, 65536, 16) == (114 * 64, 114 * 64)
+    # T=16384: 256 chunks, L = ceil(257 / 9) = 29
+    assert kda.chunk_fwd_segments(1, 16384, 16) == (29 * 64, 29 * 64)
+    # H=32, one sequence: G = 4, L = ceil(1025 / 4) = 257
+    assert kda.chunk_fwd_segments(1, 65536, 32) == (257 * 64, 257 * 64)
+    # 256 or 50 pairs (> 148 / 3): no segment scan
+    assert kda.chunk_fwd_segments(16, 4096, 16) == (0, 0)
+    assert kda.chunk_fwd_segments(1, 65536, 50) == (0, 0)
+    # packed sequences count as separate pairs: 8 sequences x 16 heads = 128 pairs
+    assert kda.chunk_fwd_segments(1, 65536, 16, 8) == (0, 0)
+    # too short to pay for the map pass: fewer than 3 segments' worth of chunks
+    assert kda.chunk_fwd_segments(1, 64, 49) == (0, 0)
+    # the product images only fit the full workspace; the minimal one runs the same plan
+    lib = kda.lib()
+    full = lib.kda_chunk_fwd_workspace(1, 65536, 16, 0, 0, 0)
+    small = lib.kda_chunk_fwd_workspace_min(1, 65536, 16, 0, 0, 0)
+    assert full - small >= 1024 * 16 * 67584 and small > 3 * 10 * 16 * 128 * 128 * 4
+    assert lib.kda_chunk_fwd_workspace(16, 4096, 16, 0, 0, 0) == lib.kda_chunk_fwd_workspace_min(16, 4096, 16, 0, 0, 0)
+
+
 def _bad_chunk(kda, **over):
     lib = kda.lib()
     a = dict(q=1 << 20, k=1 << 20, v=1 << 20, g=1 << 20, beta=1 << 20, init=None, fin=None, o=2 << 20,
