@@ -107,6 +107,32 @@ def test_varlen_with_empty_and_short_sequences(kda):
     assert eo < TOL and es < TOL, (eo, es)
 
 
+def test_varlen_mixes_whole_and_segmented_sequences(kda):
+    """Packed sequences of 100, 6000, 50 and 5850 tokens with H=4: 16 pairs, so the
+    plan cuts sequences into 6-chunk segments.  The two long sequences run through
+    the map / combine / light-output path in 16 segments each, while the two short
+    ones run whole in the first launch.  Parity against the oracle, and the same bits
+    whether the chunk products are exported or recomputed."""
+    cu = [0, 100, 6100, 6150, 12000]
+    H = 4
+    assert kda.chunk_fwd_segments(1, cu[-1], H, len(cu) - 1) == (6 * 64, 6 * 64)
+    inp = synth.op_inputs(B=len(cu) - 1, H=H, T=cu[-1], s0_std=0.02, seed=18, cu_seqlens=cu)
+    eo, es = run_both(kda, inp)
+    assert eo < TOL and es < TOL, (eo, es)
+    d = [inp[n].cuda() for n in ("q", "k", "v", "g", "beta")]
+    cu_d, s0 = inp["cu_seqlens"].cuda(), inp["s0"].cuda()
+    lib = kda.lib()
+    nseq = len(cu) - 1
+    full = lib.kda_chunk_fwd_workspace(1, cu[-1], H, nseq, 0, 0)
+    small = lib.kda_chunk_fwd_workspace_min(1, cu[-1], H, nseq, 0, 0)
+    assert small < full
+    res = [kda.chunk_fwd(*d, initial_state=s0, cu_seqlens=cu_d,
+                         workspace=torch.empty(nbytes, device="cuda", dtype=torch.uint8)) for nbytes in (full, small)]
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+
+
 def test_final_state_only_and_zero_state(kda):
     inp = synth.op_inputs(B=2, H=2, T=100, s0_std=None, seed=14)
     eo, es = run_both(kda, inp)
