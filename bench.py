@@ -459,31 +459,61 @@ def run_ours(args):
     layer = time_layer(kda, synth, dev, rank, time_calls, tc_peak, world)
     assert kda.device_status() == 0
 
-    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    # End to end through the public call with host buffers (pinned), copies inside the timed
+    # region.  Steps are pipelined as a serving loop would run them: step i+1's inputs go
+    # host -> device on their own stream while step i computes and its result comes back on a
+    # third stream (two device buffer sets, events order the reuse).  Every step still copies
+    # its own inputs in and reads its own result out.
     hq, hk, hv, hg, hb, hs0 = (t.cpu().pin_memory() for t in (q, k, v, g, beta, s0))
-    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    hfs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
-    dq, dk, dv, dg, db, ds0 = (torch.empty_like(t) for t in (q, k, v, g, beta, s0))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hs0))
-    d2h = ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size()
-    e2e_steps = max(2, min(args.steps, 5))
+    host_in = (hq, hk, hv, hg, hb, hs0)
+    host_out = [(torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                 torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)) for _ in range(2)]
+    dev_in = [[torch.empty_like(t) for t in (q, k, v, g, beta, s0)] for _ in range(2)]
+    dev_out = [(torch.empty_like(o), torch.empty_like(fs)) for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out[0][0].numel() * host_out[0][0].element_size() + host_out[0][1].numel() * host_out[0][1].element_size()
+    e2e_steps = max(2, min(args.steps, 8))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (ds0, hs0)):
-            d_.copy_(h_, non_blocking=True)
-        kda.chunk_fwd(dq, dk, dv, dg, db, initial_state=ds0, out=o, final_state=fs, workspace=ws)
-        ho.copy_(o, non_blocking=True)
-        hfs.copy_(fs, non_blocking=True)
+    def e2e_run(n):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])  # step i-2 has consumed input set b
+            with torch.cuda.stream(s_in):
+                for d_, h_ in zip(dev_in[b], host_in):
+                    d_.copy_(h_, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # step i-2's result has been read out of set b
+            dq, dk, dv, dg, db, ds0 = dev_in[b]
+            kda.chunk_fwd(dq, dk, dv, dg, db, initial_state=ds0, out=dev_out[b][0], final_state=dev_out[b][1],
+                          workspace=ws)
+            ev_comp[b].record(stream)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                host_out[b][0].copy_(dev_out[b][0], non_blocking=True)
+                host_out[b][1].copy_(dev_out[b][1], non_blocking=True)
+                ev_out[b].record(s_out)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
-    e2e_step()
+    o_ref = kda.chunk_fwd(q, k, v, g, beta, initial_state=s0, workspace=ws)[0].cpu()
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier()
     start.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps)
     end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(start.elapsed_time(end) / e2e_steps)
+    assert torch.equal(host_out[(e2e_steps - 1) & 1][0], o_ref)  # the last step's result came back
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
