@@ -217,9 +217,11 @@ int kda_dplr_chunk_fwd(const void *q, const void *k, const void *v, const void *
  * runs the same kernels, with its scratch in a static 64 MiB device array that
  * every GPU loading the library reserves until the process exits.  It never
  * allocates.
- *   - A call needing more scratch than 64 MiB (kda_chunk_fwd_workspace() of the
- *     same arguments; B=1, H=16, T=65536 bf16 needs about 31 MB) returns
- *     KDA_ERR_UNSUPPORTED without launching; use kda_chunk_fwd instead.
+ *   - It uses kda_chunk_fwd_workspace() bytes when they fit in 64 MiB; else the
+ *     kda_chunk_fwd_workspace_min() bytes, which run the same segments
+ *     recomputing the chunk products (same bits, slower); B=1, H=16, T=65536
+ *     bf16 needs about 31 MB that way.  A call needing more than 64 MiB even
+ *     then returns KDA_ERR_UNSUPPORTED without launching; use kda_chunk_fwd.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls share the array: calls whose kernels can overlap on the GPU
