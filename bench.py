@@ -33,12 +33,7 @@ GDN_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + 4 + 4  # q,k,v + o (bf16), one fp
 FLOP_PER_TOKEN_HEAD = 6 * D * D + 3 * 64 * D + 64 * 64  # the pages' per-head count, C = 64
 
 
-def metric_name():
-    try:
-        with open(os.path.join(ROOT, "BASELINE.json")) as f:
-            return json.load(f)["metric"]
-    except Exception:
-        return "KDA prefill tokens/s (H=16,T=64K) + decode state GB/s, % of B200 roofline"
+METRIC = "KDA prefill tokens/s (H=16,T=64K) + decode state GB/s, % of B200 roofline"
 
 
 def profiled_traffic(summary: str, source: str):
@@ -180,7 +175,7 @@ def run_reference(args):
     t = statistics.mean(times)
     value = T_s / t  # tokens/s with all 16 heads of each token
     line = {
-        "metric": metric_name(), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"KDA prefill B=1 H=16 d=128, oracle sample of {T_s} tokens x {H_s} heads per step",
@@ -359,7 +354,7 @@ def run_ours(args):
 
     if args.prefill_only:
         if rank == 0:
-            print(json.dumps({"metric": metric_name(), "value": value, "unit": "tokens/s", "ms_per_step": ms,
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms,
                               "config": {"workload": f"KDA prefill B=1 H=16 T={T} (prefill only)", "timing": timing},
                               "roofline": roofline}), flush=True)
         ranks.close()
@@ -524,7 +519,7 @@ def run_ours(args):
 
     if rank == 0:
         line = {
-            "metric": metric_name(), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"KDA prefill B=1 H=16 T={T} d=128 bf16, fp32 g/beta/state "

@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,  /* NULL where not allowed, bad size, misaligned pointer */
-    KDA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. head dim != 128) */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid request this library does not implement (e.g. head dim != 128) */
     KDA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than the matching *_workspace() query */
     KDA_ERR_CUDA = 4,         /* a CUDA runtime / driver call or kernel launch failed */
     KDA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see kda_device_status) */
@@ -61,7 +61,7 @@ typedef enum {
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *kda_status_string(int status);
 
-/* Head dimension this build supports (d_k = d_v): 128. */
+/* Head dimension this library supports (d_k = d_v): 128. */
 int kda_head_dim(void);
 
 /* Detail of the last host-side rejection or CUDA error on this thread
@@ -290,7 +290,7 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
  * (sequence, head) runs the forward once storing the state every 64 tokens,
  * then walks the chunks backwards, recomputing each chunk's states.  It is the
  * reference-speed backward (about 2x the token-serial forward work per token);
- * a chunked tensor-core backward is not part of this build.
+ * a chunked tensor-core backward is not part of this library.
  *
  *   q, k, v, d_o   [B,T,H,128], dtype bf16 or fp32 (q, k not normalised here).
  *   g              fp32 [B,T,H,128];  beta fp32 [B,T,H].
