@@ -1476,15 +1476,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
 // Chains the segment maps of one (sequence, head, 16-column slice):
 // S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1 (segment 0
 // gets the initial state).  X_g^T (64 KB, written transposed by the summary
-// pass) streams into shared memory with 1-D bulk copies, double-buffered; each
-// thread owns a 2 x 4 tile of the slice.
+// pass) streams into shared memory with 1-D bulk copies, double-buffered.  Two
+// halves of 256 threads each sum over half of the key dimension, a thread owning
+// a 2 x 4 tile of the slice; the halves' sums meet in shared memory.
 constexpr int kCombCols = 16;
-constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 64;
+constexpr int kCombThreads = 512;  // two halves of 256, each summing over half of the key dimension
+constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 256 * 8 * 4 + 64;
 
 
-__global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, const int* n_items, const int* seq_first,
-                                                      int N, const float* init, const float* segN,
-                                                      const float* segXt, float* segS, int H) {
+__global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem* items, const int* n_items,
+                                                                  const int* seq_first, int N, const float* init,
+                                                                  const float* segN, const float* segXt,
+                                                                  float* segS, int H) {
     const int n = blockIdx.x, h = blockIdx.y, z = blockIdx.z;  // one CTA per (sequence, head, slice)
     if (n >= N) return;
     const int item = seq_first[n];
@@ -1494,9 +1497,11 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, c
     extern __shared__ __align__(128) uint8_t csm[];
     float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
     float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(csm + 2 * 65536 + kD * kCombCols * 4);  // [2]
-    const int tid = threadIdx.x;
-    const int k0 = (tid >> 2) * 2, j0 = (tid & 3) * 4;  // rows k0, k0+1; cols j0..j0+3 of the slice
+    float* sR = sS + kD * kCombCols;                                 // [256][8] the upper half's partial sums
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sR + 256 * 8);       // [2]
+    const int tid = threadIdx.x, half = tid >> 8, t = tid & 255;
+    const int k0 = (t >> 2) * 2, j0 = (t & 3) * 4;  // rows k0, k0+1; cols j0..j0+3 of the slice
+    const int kp0 = half * (kD / 2);                 // this half's key range [kp0, kp0 + 64)
     const int c0 = kCombCols * z;
     const size_t hs = size_t(h) * (kD * kD);
     if (tid == 0) {
@@ -1511,7 +1516,7 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, c
         bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + j) * H * (kD * kD) + hs, 65536u, &bar[j & 1]);
     };
     if (tid == 0) fetch(0);
-    for (int e = tid; e < kD * kCombCols; e += 256) {
+    for (int e = tid; e < kD * kCombCols; e += kCombThreads) {
         const int kk = e / kCombCols, jj = e % kCombCols;
         sS[e] = init ? init[size_t(it.seq) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] : 0.f;
     }
@@ -1527,15 +1532,16 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, c
         const size_t base = size_t(item + g) * H * (kD * kD) + hs;
         float acc[2][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {  // N_g's slice: requested before the wait for X_g
-            const float4 n4 = *reinterpret_cast<const float4*>(segN + base + size_t(k0 + r) * kD + c0 + j0);
+        for (int r = 0; r < 2; ++r) {  // the lower half starts from N_g's slice (requested before the wait)
+            float4 n4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (half == 0) n4 = *reinterpret_cast<const float4*>(segN + base + size_t(k0 + r) * kD + c0 + j0);
             acc[r][0] = n4.x; acc[r][1] = n4.y; acc[r][2] = n4.z; acc[r][3] = n4.w;
         }
         ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
         if (__syncthreads_or(!ok)) break;
         const float* X = sX + (j & 1) * kD * kD;
 #pragma unroll 1
-        for (int kb = 0; kb < kD; kb += 8) {  // acc[k][j] += X[k][kp] S[kp][j] = Xt[kp][k] S[kp][j]
+        for (int kb = kp0; kb < kp0 + kD / 2; kb += 8) {  // acc[k][j] += Xt[kp][k] S[kp][j]
             float2 xv[8];  // 8 key steps' operands requested before their FMAs (hides the load latency)
             float4 sv[8];
 #pragma unroll
@@ -1551,13 +1557,22 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(const SegItem* items, c
                 acc[1][2] += xv[u].y * sv[u].z; acc[1][3] += xv[u].y * sv[u].w;
             }
         }
-        __syncthreads();  // every thread has read sS and this X buffer
-        const size_t out = size_t(item + g + 1) * H * (kD * kD) + hs;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const float4 v4 = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-            *reinterpret_cast<float4*>(sS + (k0 + r) * kCombCols + j0) = v4;
-            *reinterpret_cast<float4*>(segS + out + size_t(k0 + r) * kD + c0 + j0) = v4;
+        if (half == 1) {
+            float4* r4 = reinterpret_cast<float4*>(sR + t * 8);
+            r4[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+            r4[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+        }
+        __syncthreads();  // every thread has read sS and this X buffer; the upper half's sums are in sR
+        if (half == 0) {
+            const float4* r4 = reinterpret_cast<const float4*>(sR + t * 8);
+            const float4 p0 = r4[0], p1 = r4[1];
+            const size_t out = size_t(item + g + 1) * H * (kD * kD) + hs;
+            const float4 v0 = make_float4(acc[0][0] + p0.x, acc[0][1] + p0.y, acc[0][2] + p0.z, acc[0][3] + p0.w);
+            const float4 v1 = make_float4(acc[1][0] + p1.x, acc[1][1] + p1.y, acc[1][2] + p1.z, acc[1][3] + p1.w);
+            *reinterpret_cast<float4*>(sS + k0 * kCombCols + j0) = v0;
+            *reinterpret_cast<float4*>(sS + (k0 + 1) * kCombCols + j0) = v1;
+            *reinterpret_cast<float4*>(segS + out + size_t(k0) * kD + c0 + j0) = v0;
+            *reinterpret_cast<float4*>(segS + out + size_t(k0 + 1) * kD + c0 + j0) = v1;
         }
         __syncthreads();
     }
@@ -1808,7 +1823,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                 return KDA_ERR_CUDA;
             comb_attr = true;
         }
-        combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), 256, kCombSmem, stream>>>(
+        combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), kCombThreads, kCombSmem, stream>>>(
             items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) trace_record(ev[3], stream);
         const int r2 = launch_phase_for<2>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
