@@ -28,7 +28,7 @@ SYMBOLS = (
     "kda_layer_fwd_workspace", "kda_layer_fwd", "kda_set_trace_events", "kda_chunk_fwd_noalloc",
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
     "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
-    "kda_chunk_fwd_segment_tokens", "kda_chunk_fwd_workspace_min",
+    "kda_chunk_fwd_segment_tokens", "kda_chunk_fwd_workspace_min", "kda_debug_fault_injection",
 )
 
 
@@ -85,6 +85,8 @@ def _load():
     lib.kda_layer_decode_workspace.restype = sz
     lib.kda_layer_decode.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, vp, vp, i, i, vp, sz, vp]
     lib.kda_layer_decode.restype = i
+    lib.kda_debug_fault_injection.argtypes = [ctypes.c_longlong, i]
+    lib.kda_debug_fault_injection.restype = i
     lib.kda_set_trace_events.argtypes = [vp, i]
     lib.kda_set_trace_events.restype = i
     return lib
@@ -122,6 +124,13 @@ def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
     return _lib.kda_device_status(s)
+
+
+def debug_fault_injection(wait_limit_cycles=0, skip_chunk=-1):
+    """Failure-test hook (``kda_debug_fault_injection``): bound of every device-side
+    wait in SM cycles (0 = the default) and a chunk whose input load the chunk
+    kernels skip (-1 = none).  Device-global; for tests only."""
+    _check(_lib.kda_debug_fault_injection(int(wait_limit_cycles), int(skip_chunk)), "kda_debug_fault_injection")
 
 
 def set_trace_events(events):

@@ -91,6 +91,15 @@ int kda_device_status(void* stream) {
     return KDA_OK;
 }
 
+int kda_debug_fault_injection(long long wait_limit_cycles, int skip_chunk) {
+    t_last_error[0] = 0;
+    const long long lim = wait_limit_cycles > 0 ? wait_limit_cycles : (1ll << 31);
+    const int skip = skip_chunk >= 0 ? skip_chunk : -1;
+    cudaError_t e = cudaMemcpyToSymbol(c_wait_limit, &lim, sizeof(lim));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_skip_chunk_load, &skip, sizeof(skip));
+    return e == cudaSuccess ? KDA_OK : fail(KDA_ERR_CUDA, cudaGetErrorString(e));
+}
+
 int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int* middle_tokens) {
     if (middle_tokens) *middle_tokens = 0;
     if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;

@@ -279,7 +279,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     const int t_begin = it.tok_begin, t_end = it.tok_end;
     const int nchunks = (t_end - t_begin + kC - 1) / kC;
 
-    auto issue_qkg = [&](int c) {
+    auto issue_qkg = [&](int c) -> bool {  // false: skipped by the failure-test hook
+        if (c == c_skip_chunk_load) return false;
         const int t0 = t_begin + c * kC;
         mbar_arrive_expect_tx(&bars[0], 65536u - (kScalarGate ? 32768u : 0u));
         tma_load_3d(sm + OFF_Q, &tm_q, &bars[0], 0, h, t0);
@@ -287,6 +288,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         tma_load_3d(sm + OFF_K, &tm_k, &bars[0], 0, h, t0);
         tma_load_3d(sm + OFF_K + 8192, &tm_k, &bars[0], 64, h, t0);
         if (!kScalarGate) tma_load_3d(sm + OFF_G, &tm_g, &bars[0], 0, h, t0);
+        return true;
     };
     auto issue_v = [&](int c) {
         const int t0 = t_begin + c * kC;
@@ -296,9 +298,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     };
     bool pend_qkg = false, pend_v = false;  // meaningful in the loader thread only
     if (tid == kLoader && nchunks > 0) {
-        issue_qkg(0);
+        pend_qkg = issue_qkg(0);
         issue_v(0);
-        pend_qkg = pend_v = true;
+        pend_v = true;
     }
 
     // ---- start state into TMEM: S^T (lane = v, column = k); X^T = I for the summary.
@@ -561,8 +563,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             fence_async_smem();
             __syncthreads();
             if (fast_next && tid == kLoader && nchunks > 1) {  // q, k, g of chunk 0 are consumed
-                issue_qkg(1);
-                pend_qkg = true;
+                pend_qkg = issue_qkg(1);
             }
         }
     }
@@ -725,8 +726,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             }
             __syncthreads();  // the q / k / b tiles are read
             if (tid == kLoader && c + 1 < nchunks) {
-                issue_qkg(c + 1);
-                pend_qkg = true;
+                pend_qkg = issue_qkg(c + 1);
             }
             for (int e = tid; e < 64 * 64; e += kThreads) sA[e] = 0.f;
             for (int e = tid; e < 512; e += kThreads) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
@@ -1088,8 +1088,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             bulk_commit();
         }
         if (has_next && fast_next && tid == kLoader && c + 2 < nchunks) {  // q, k, g of chunk c+1 are consumed
-            issue_qkg(c + 2);
-            pend_qkg = true;
+            pend_qkg = issue_qkg(c + 2);
         }
         KDA_STAGE(13);
     }
@@ -1695,12 +1694,7 @@ template <int kPhase, typename O, bool G>
 static int launch_phase(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a, cudaStream_t stream) {
     auto kern = kPhase == 1 ? chunk_phase1_kernel<O, G> : chunk_phase2_kernel<O, G>;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr = true;
-    }
+    if (!set_smem_attr(kern, kSmemBytes)) return KDA_ERR_CUDA;
     kern<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
     return KDA_OK;
 }
@@ -1816,13 +1810,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     if (r1 != KDA_OK) return r1;
     if (pl.scan) {
         if (ev) trace_record(ev[2], stream);
-        static bool comb_attr = false;
-        if (!comb_attr) {
-            if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombSmem) !=
-                cudaSuccess)
-                return KDA_ERR_CUDA;
-            comb_attr = true;
-        }
+        if (!set_smem_attr(combine_kernel, kCombSmem)) return KDA_ERR_CUDA;
         combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), kCombThreads, kCombSmem, stream>>>(
             items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) trace_record(ev[3], stream);

@@ -28,6 +28,15 @@ constexpr int kC = 64;       // chunk length
 // translation unit (kda_lib.cu), so this is its only definition.
 __device__ int g_device_status = 0;
 
+// Bound of every device-side wait, in SM cycles: 2^31 by default (about a
+// second at the B200's clock).  kda_debug_fault_injection() lowers it for the
+// failure tests.
+__constant__ long long c_wait_limit = 1ll << 31;
+// Chunk (index inside a launch's sequence segment) whose q/k/g load the chunk
+// kernels' loader skips, or -1.  Set only by kda_debug_fault_injection() for
+// the failure tests: the bounded wait for the skipped load then gives up.
+__constant__ int c_skip_chunk_load = -1;
+
 __device__ __forceinline__ void report_timeout(int where) {
     atomicOr(&g_device_status, 1 << (where & 15));
 }
@@ -58,15 +67,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait on a phase of an mbarrier.  Gives up after ~2^31 SM cycles
-// (about a second) and returns false; the caller then aborts cleanly.
+// Bounded wait on a phase of an mbarrier.  Gives up after c_wait_limit SM
+// cycles (default 2^31, about a second) or 2^26 polls, whichever comes first,
+// records the site bit and returns false; the caller then aborts cleanly.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
-    const long long t0 = clock64();
+    const long long t0 = clock64(), limit = c_wait_limit;
     for (uint32_t it = 0; it < (1u << 26); ++it) {
         if (mbar_try_wait(a, parity)) return true;
-        if (clock64() - t0 > (1ll << 31)) break;
+        if (clock64() - t0 > limit) break;
     }
     report_timeout(where);
     return false;
@@ -196,6 +206,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- misc
+// Lets a kernel launch with `bytes` of dynamic shared memory (above the 48 KB
+// default).  The attribute belongs to the current device's context, so it is
+// set before every launch: a cheap host call that stays right on a second GPU
+// of the same process and after a device reset.
+template <typename Kern>
+inline bool set_smem_attr(Kern kern, uint32_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) == cudaSuccess;
+}
+
 // Two fp32 -> packed bf16x2, rounding to nearest on the bit pattern (ties away
 // from zero) with integer ops: adding half an ulp of bf16 (0x8000) to the fp32
 // bits and keeping the top half.  This keeps the packing on the integer pipe

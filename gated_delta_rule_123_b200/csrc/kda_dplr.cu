@@ -731,12 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <typename O>
 static cudaError_t dplr_smem_attr() {
-    static bool done = false;
-    if (done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(dplr_chunk_kernel<O>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         dplr::kSmem);
-    if (e == cudaSuccess) done = true;
-    return e;
+    return set_smem_attr(dplr_chunk_kernel<O>, dplr::kSmem) ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 size_t dplr_workspace_bytes(int B, int T, int H, int num_seqs, int dtype) {

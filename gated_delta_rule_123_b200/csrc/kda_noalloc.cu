@@ -10,10 +10,12 @@
 // The array is kNoAllocScratchBytes per GPU, reserved on every device that
 // loads this library and held until the process exits.  Host code cannot pass
 // the array's name to a kernel (on the host it is only a stand-in, not a device
-// address), so the device address is looked up with cudaGetSymbolAddress once
-// per device, with that device current, on the first call made on it.  That
-// first call on a device therefore does a little host-side set-up and should
-// come before any stream capture.  Nothing here calls cudaMalloc, cudaFree or
+// address), so each call looks the device address up with cudaGetSymbolAddress
+// on the current device.  Once the library's device code is loaded on a device
+// that is a host-side table lookup; the first call on a device loads it, so
+// that first call should come before any stream capture.  Looking the address
+// up on every call (rather than caching it) keeps it right after a device
+// reset, which can move the array.  Nothing here calls cudaMalloc, cudaFree or
 // any allocating library routine.
 //
 // All calls share the one array: two calls whose kernels overlap on the GPU
@@ -22,40 +24,26 @@
 // array keeps the last call's contents; the chunk path writes every scratch
 // word it reads (segment table, segment states) before reading it, so nothing
 // needs clearing between calls.
-#include <mutex>
-
 #include "kda_common.cuh"
 
 namespace kda {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
-constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 
-// Device address of g_noalloc_scratch on the current device (looked up once).
+// Device address of g_noalloc_scratch on the current device.
 static void* noalloc_scratch(const char** why) {
-    static std::mutex mu;
-    static void* addr[kNoAllocMaxDevices] = {};
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
-        *why = "no usable current CUDA device";
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+        *why = e != cudaSuccess ? cudaGetErrorString(e) : "no device address for the static scratch array";
         return nullptr;
     }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || p == nullptr) {
-            *why = cudaGetErrorString(e);
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace kda

@@ -73,6 +73,20 @@ const char *kda_last_error(void);
  * up a bounded wait since the last call, or KDA_ERR_CUDA if the sync failed. */
 int kda_device_status(void *stream);
 
+/* Testing hook for the failure path of the bounded device-side waits (no
+ * counterpart on the pages).  wait_limit_cycles > 0 sets the bound of every
+ * later device-side wait of this library on the current device, in SM cycles;
+ * <= 0 restores the default of 2^31 (about a second).  skip_chunk >= 0 makes
+ * every later launch of the chunk kernels' map/whole-sequence pass skip the
+ * q/k/g load of that chunk (counted inside the launch's sequence segment) of
+ * each (sequence, head): the wait for it then gives up, the kernel records
+ * KDA_ERR_TIMEOUT in the device status word and exits cleanly, without a trap
+ * or a hang, and that call's results are undefined.  skip_chunk < 0 turns the
+ * skip off.  The settings are global to the device: change them only while no
+ * call of this library runs.  Synchronous (legacy default stream).  Production
+ * code never needs it. */
+int kda_debug_fault_injection(long long wait_limit_cycles, int skip_chunk);
+
 /* Optional tracing hook for kda_chunk_fwd.  When `events` is non-NULL it must
  * point to 5 cudaEvent_t created by the caller on the current device; every
  * later kda_chunk_fwd call on this thread records them on its stream around
@@ -122,7 +136,10 @@ int kda_set_trace_events(void *events, int n_events);
  *
  * Tensor cores compute the chunk contractions with bf16 operands and fp32
  * accumulation; the state is carried in fp32.  fp32 inputs are rounded to
- * bf16 where they feed the tensor cores.
+ * bf16 where they feed the tensor cores.  Rounding: a bf16 o is rounded from
+ * its fp32 accumulator once, to nearest with ties to even; the bf16 operands
+ * the kernels form on chip (gated keys and queries, W, U~, the state copy) are
+ * rounded to nearest with ties away from zero.
  */
 /* How a kda_chunk_fwd call with these sizes on the current device is split:
  * 0 when every (sequence, head) runs in one CTA; otherwise the length in tokens
@@ -222,8 +239,10 @@ int kda_dplr_chunk_fwd(const void *q, const void *k, const void *v, const void *
  *     recomputing the chunk products (same bits, slower); B=1, H=16, T=65536
  *     bf16 needs about 31 MB that way.  A call needing more than 64 MiB even
  *     then returns KDA_ERR_UNSUPPORTED without launching; use kda_chunk_fwd.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress: a host-side lookup once the library's device code
+ *     is loaded there, and still right after a device reset).  The first call
+ *     on a device loads that code; make it before any stream capture.
  *   - All calls share the array: calls whose kernels can overlap on the GPU
  *     (e.g. on two unordered streams) race and corrupt each other's results.
  *     Calls ordered on one stream are safe; nothing needs clearing between them.
