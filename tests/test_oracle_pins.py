@@ -311,3 +311,61 @@ def test_layer_packed_equals_separate():
         yn, sn = L.kda_layer(x[t0:t1], W, [0, t1 - t0], H=2)
         np.testing.assert_allclose(y[t0:t1], yn, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(s[n], sn[0], rtol=1e-12, atol=1e-14)
+
+
+# --- 12. hand-derived golden example of the layer --------------------------------------
+def _load_layer_golden():
+    """Evaluate tests/golden/kda_layer_tiny.txt line by line (closed forms derived by
+    hand; silu and sigmoid are torch's, log and sqrt are math's)."""
+    import math
+
+    def _f(fn):
+        return lambda u: float(fn(torch.tensor(float(u), dtype=torch.float64)))
+
+    ns = {"log": math.log, "sqrt": math.sqrt, "silu": _f(torch.nn.functional.silu), "sigmoid": _f(torch.sigmoid),
+          "vec": lambda *a: np.array(a, dtype=np.float64)}
+    with open(os.path.join(GOLDEN, "kda_layer_tiny.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            name, expr = (s.strip() for s in line.split("=", 1))
+            ns[name] = eval(expr, {"__builtins__": {}}, ns)  # noqa: S307 (a committed test fixture)
+    return ns
+
+
+_LAYER_WEIGHTS = ("W_q", "W_k", "W_v", "conv_q", "conv_k", "conv_v", "W_adown", "W_aup", "W_gdown", "W_gup",
+                  "W_b", "norm_w", "W_o")
+
+
+def test_layer_golden_tiny_example():
+    """The layer's assembly, stage by stage, against a hand-derived example: q, k
+    after ShortConv, SiLU and the per-head L2 norm; v; the decay alpha; beta; the
+    output gate; then y and the final state through the recurrence, the per-head
+    RMSNorm times the gate and the output projection."""
+    from oracle import layer as L
+    ns = _load_layer_golden()
+    W = {n: np.array(ns[n], dtype=np.float64) for n in _LAYER_WEIGHTS}
+    x, cu = np.array(ns["x"], dtype=np.float64), ns["cu"]
+    q, k, v, g, beta, gate = L.layer_reference_parts(x, W, cu, 2)
+    np.testing.assert_allclose(q, np.array(ns["q"]), atol=1e-13)
+    np.testing.assert_allclose(k, np.array(ns["k"]), atol=1e-13)
+    np.testing.assert_allclose(v, np.array(ns["v"]), atol=1e-13)
+    np.testing.assert_allclose(np.exp(g), np.array(ns["alpha"]), atol=1e-13)
+    np.testing.assert_allclose(beta, np.array(ns["beta"]), atol=1e-13)
+    np.testing.assert_allclose(L.sigmoid(gate), np.array(ns["sg"]), atol=1e-13)
+    y, S = oracle.kda_layer(x, W, cu, 2, s0=np.array(ns["S0"], dtype=np.float64))
+    np.testing.assert_allclose(S, np.array(ns["S_final"]), atol=1e-13)
+    np.testing.assert_allclose(y, np.array(ns["y"]), atol=1e-12)
+
+
+@pytest.mark.parametrize("swap", [("W_q", "W_k"), ("conv_q", "conv_k")])
+def test_layer_golden_detects_swapped_projections(swap):
+    """The example is asymmetric: the same oracle fed W_q and W_k (or the q and k
+    convolution taps) the other way round misses the hand-derived y."""
+    ns = _load_layer_golden()
+    W = {n: np.array(ns[n], dtype=np.float64) for n in _LAYER_WEIGHTS}
+    W[swap[0]], W[swap[1]] = W[swap[1]], W[swap[0]]
+    y, _ = oracle.kda_layer(np.array(ns["x"], dtype=np.float64), W, ns["cu"], 2,
+                            s0=np.array(ns["S0"], dtype=np.float64))
+    assert np.abs(y - np.array(ns["y"])).max() > 1e-2
