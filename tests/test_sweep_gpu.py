@@ -8,8 +8,9 @@ length, B=1, 16 heads, up to 64K).
 
 Every length runs in the launch configuration the bench would time (the
 segment plan cuts each length differently: ``kda_chunk_fwd_segment_tokens``).
-The oracle checks three sampled heads end to end: relative L2 <= 1e-2 on o and
-on the final state, as for every prefill test."""
+The oracle checks three sampled heads end to end (one for the untied DPLR
+kernel, whose product-form oracle costs O(d^3) per token): relative L2 <= 1e-2
+on o and on the final state, as for every prefill test."""
 import numpy as np
 import pytest
 import torch
@@ -79,5 +80,6 @@ def test_dplr_sweep_sampled_heads(kda, T):
     def ref(a, s0):
         return oracle.dplr_recurrent(a["q"], a["k"], a["v"], a["g"], a["beta"], a["a"], a["b"], s0=s0)
 
-    eo, es = _check(o, fs, inp, torch.tensor(HEADS), ref)
+    # the product-form DPLR oracle costs O(d^3) per token: one sampled head
+    eo, es = _check(o, fs, inp, torch.tensor([HEADS[1]]), ref)
     assert eo < TOL and es < TOL, (eo, es)
