@@ -204,11 +204,23 @@ def time_layer(kda, synth, dev, rank, time_calls, tc_peak, world):
     HDl, dm, rk = lc["H"] * D, lc["d_model"], lc["rank"]
     gemm_flop = 2 * lc["Ttot"] * (dm * (3 * HDl + 2 * rk + lc["H"]) + 2 * rk * HDl + HDl * dm)
     flop = gemm_flop + FLOP_PER_TOKEN_HEAD * lc["Ttot"] * lc["H"]
+    # the two large projections alone, through kda_linear_bf16 (the layer's GEMM kernel)
+    gemms = {}
+    for name, n_out, k_in, w in (("input_projection", lpk["W_in"].shape[0], dm, lpk["W_in"]),
+                                  ("output_projection", dm, HDl, lpk["W_o"])):
+        a = torch.randn((lc["Ttot"], k_in), device=dev, generator=torch.Generator(device=dev).manual_seed(9)
+                        ).to(torch.bfloat16)
+        yo = torch.empty((lc["Ttot"], (n_out + 7) // 8 * 8), device=dev, dtype=torch.bfloat16)[:, :n_out]
+        gms = time_calls(lambda: kda.linear(a, w, out=yo), 10)
+        gf = 2 * lc["Ttot"] * n_out * k_in
+        gemms[name] = {"M": lc["Ttot"], "N": n_out, "K": k_in, "ms": gms, "tflops": gf / (gms / 1e3) / 1e12,
+                       "frac": gf / (gms / 1e3) / 1e12 / tc_peak}
+        del a, yo
     return {"workload": "KDA layer d_model=2048 H=16 rank=128, 65536 packed tokens (8 sequences), "
                         "random-init bf16 weights", "ms_per_call": ms,
             "tokens_per_s": world * lc["Ttot"] / (ms / 1e3), "tflops": flop / (ms / 1e3) / 1e12,
             "gemm_tflop_per_call": gemm_flop / 1e12, "tensor_peak_tflops": tc_peak,
-            "frac": flop / (ms / 1e3) / 1e12 / tc_peak}
+            "frac": flop / (ms / 1e3) / 1e12 / tc_peak, "gemm": gemms}
 
 
 def run_ours(args):

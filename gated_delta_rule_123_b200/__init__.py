@@ -29,6 +29,7 @@ SYMBOLS = (
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
     "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
     "kda_chunk_fwd_segment_tokens", "kda_chunk_fwd_workspace_min", "kda_debug_fault_injection",
+    "kda_linear_bf16",
 )
 
 
@@ -85,6 +86,8 @@ def _load():
     lib.kda_layer_decode_workspace.restype = sz
     lib.kda_layer_decode.argtypes = [vp, ctypes.POINTER(LayerWeights), vp, vp, vp, i, i, vp, sz, vp]
     lib.kda_layer_decode.restype = i
+    lib.kda_linear_bf16.argtypes = [vp, i, vp, i, vp, i, i, i, i, vp]
+    lib.kda_linear_bf16.restype = i
     lib.kda_debug_fault_injection.argtypes = [ctypes.c_longlong, i]
     lib.kda_debug_fault_injection.restype = i
     lib.kda_set_trace_events.argtypes = [vp, i]
@@ -278,6 +281,21 @@ def recurrent_fwd(q, k, v, g, beta, state, scale=1.0, l2norm_qk=False, out=None)
                                 _dtype_code(q), float(scale), int(l2norm_qk), _stream(q.device))
     _check(rc, "kda_recurrent_fwd")
     return o
+
+
+def linear(x, W, out=None):
+    """y = x W^T (``kda_linear_bf16``): x [M, K] and W [N, K] bf16 with contiguous rows.
+    Returns y [M, N] bf16 (a view with a row stride padded to 8 elements when N is not
+    a multiple of 8)."""
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K or x.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise ValueError("linear: x [M, K] and W [N, K] must be bf16")
+    y = out if out is not None else torch.empty((M, (N + 7) // 8 * 8), device=x.device, dtype=torch.bfloat16)[:, :N]
+    rc = _lib.kda_linear_bf16(_ptr(x), x.stride(0), _ptr(W), W.stride(0), _ptr(y), y.stride(0), M, N, K,
+                              _stream(x.device))
+    _check(rc, "kda_linear_bf16")
+    return y
 
 
 def pack_layer_weights(W: dict) -> dict:

@@ -37,7 +37,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp,
-           os.path.join(CSRC, "kda_lib.cu"), "-lcublasLt"]
+           os.path.join(CSRC, "kda_lib.cu")]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)

@@ -3,7 +3,7 @@
 #include <stdio.h>
 #include <string.h>
 
-#include "kda_common.cuh"
+#include "kda_gemm.cuh"
 
 namespace kda {
 
@@ -21,13 +21,13 @@ int chunk_segment_tokens(int B, int T, int H, int num_seqs, int* middle);
 size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
-                         cudaStream_t stream);
+                         cudaStream_t stream, int out_f32);
 int launch_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                        float* state, void* o, int B, int H, int dtype, float scale, int l2norm, cudaStream_t stream);
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why, int scalar_gate);
+                     const char** why, int scalar_gate, int out_f32);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 size_t layer_workspace_bytes(int total_tokens, int d_model, int H, int rank, int num_seqs);
 int launch_layer_fwd(const void* x, const kda_layer_weights* w, const int32_t* cu, int nseq, int ntok,
@@ -158,7 +158,7 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
     const char* why = "";
     const int rc = launch_chunk_fwd(q, k, v, g, beta, initial_state, final_state, o, cu_seqlens, num_seqs, B, T, H,
                                     dtype, scale, l2norm_qk, workspace, workspace_bytes,
-                                    static_cast<cudaStream_t>(stream), &why, scalar_gate);
+                                    static_cast<cudaStream_t>(stream), &why, scalar_gate, 0);
     return rc == KDA_OK ? KDA_OK : fail(rc, why);
 }
 
@@ -293,8 +293,25 @@ int kda_recurrent_fwd(const void* q, const void* k, const void* v, const float* 
         return fail(KDA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if (o == q || o == k || o == v) return fail(KDA_ERR_INVALID_ARG, "o must not alias q, k or v");
     const int rc = launch_recurrent_fwd(q, k, v, g, beta, state, o, B, T, H, dtype, scale, l2norm_qk,
-                                        static_cast<cudaStream_t>(stream));
+                                        static_cast<cudaStream_t>(stream), 0);
     return rc == KDA_OK ? KDA_OK : fail(rc, cudaGetErrorString(cudaGetLastError()));
+}
+
+int kda_linear_bf16(const void* x, int ldx, const void* W, int ldw, void* y, int ldy, int M, int N, int K,
+                    void* stream) {
+    t_last_error[0] = 0;
+    if (M < 0 || N < 0 || K < 0) return fail(KDA_ERR_INVALID_ARG, "negative size");
+    if ((long long)M * N == 0) return KDA_OK;
+    if (K == 0) return fail(KDA_ERR_UNSUPPORTED, "K must be positive");
+    if (!x || !W || !y) return fail(KDA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (ldx < K || ldw < K || ldy < N) return fail(KDA_ERR_INVALID_ARG, "row stride smaller than the row");
+    if (!aligned16(x) || !aligned16(W) || !aligned16(y) || ldx % 8 || ldw % 8 || ldy % 8)
+        return fail(KDA_ERR_INVALID_ARG, "pointers and row strides must be 16-byte aligned");
+    if (y == x || y == W) return fail(KDA_ERR_INVALID_ARG, "y must not alias x or W");
+    const char* why = "";
+    const int rc = launch_gemm(x, ldx, W, ldw, y, ldy, M, N, K, GemmEpilogue{}, static_cast<cudaStream_t>(stream),
+                               &why);
+    return rc == KDA_OK ? KDA_OK : fail(rc, why);
 }
 
 size_t kda_layer_fwd_workspace(int total_tokens, int d_model, int H, int rank, int num_seqs) {

@@ -1721,10 +1721,12 @@ static inline void trace_record(cudaEvent_t e, cudaStream_t stream) {
         cudaEventRecord(e, stream);
 }
 
+// out_f32 != 0 writes o in fp32 whatever the input dtype (the layer's use).
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why, int scalar_gate) {
+                     const char** why, int scalar_gate, int out_f32) {
+    const int out_dtype = (dtype == KDA_FP32 || out_f32) ? KDA_FP32 : KDA_BF16;
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
     // A workspace of kda_chunk_fwd_workspace() bytes holds the exported chunk products of
     // segmented calls; one of only total_min bytes runs the same schedule recomputing them.
@@ -1774,7 +1776,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         !make_map(&mg, scalar_gate ? kb : g, scalar_gate ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                   scalar_gate ? 2 : 4, H, Tmap, scalar_gate ? 64 : 128,
                   scalar_gate ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mo, dtype == KDA_FP32 ? vb : o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64,
+        !make_map(&mo, out_dtype == KDA_FP32 ? vb : o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, Tmap, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "cuTensorMapEncodeTiled failed";
         return KDA_ERR_CUDA;
@@ -1806,7 +1808,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         trace_record(ev[2], stream);
         trace_record(ev[3], stream);
     }
-    const int r1 = launch_phase_for<1>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
+    const int r1 = launch_phase_for<1>(out_dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
     if (r1 != KDA_OK) return r1;
     if (pl.scan) {
         if (ev) trace_record(ev[2], stream);
@@ -1814,7 +1816,7 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), kCombThreads, kCombSmem, stream>>>(
             items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
         if (ev) trace_record(ev[3], stream);
-        const int r2 = launch_phase_for<2>(dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
+        const int r2 = launch_phase_for<2>(out_dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
         if (r2 != KDA_OK) return r2;
     }
     if (ev) trace_record(ev[4], stream);

@@ -153,11 +153,11 @@ int launch_decode_step(const void* q, const void* k, const void* v, const float*
 // are double-buffered.  Buffer reuse distances: a token buffer written during
 // token t (for t+1) was last read during token t-2, and every warp has passed
 // token t-1's barrier before any warp starts token t.
-template <typename T>
+template <typename T, typename OutT>
 __global__ void __launch_bounds__(256, 2)
     recurrent_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                          const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
-                         T* __restrict__ o, int Tn, int H, float scale, int l2norm) {
+                         OutT* __restrict__ o, int Tn, int H, float scale, int l2norm) {
     __shared__ __align__(16) float sk[3][kD], sq[3][kD], sa[3][kD], sv[3][kD];
     __shared__ float sdot[3][4][3];  // per loader warp: k.k, q.q, k.q
     __shared__ float sb[3];
@@ -257,11 +257,11 @@ __global__ void __launch_bounds__(256, 2)
         u.w = bt * (v4.w - ys.w);
         if (warp == 0) {  // o = S_new^T q = z + (k^T q) u, scales folded in
             const float c = kq * nk * nq;
-            T* op = o + row(t) * kD + 4 * lane;
-            op[0] = from_f32<T>(zs.x + c * u.x);
-            op[1] = from_f32<T>(zs.y + c * u.y);
-            op[2] = from_f32<T>(zs.z + c * u.z);
-            op[3] = from_f32<T>(zs.w + c * u.w);
+            OutT* op = o + row(t) * kD + 4 * lane;
+            op[0] = from_f32<OutT>(zs.x + c * u.x);
+            op[1] = from_f32<OutT>(zs.y + c * u.y);
+            op[2] = from_f32<OutT>(zs.z + c * u.z);
+            op[3] = from_f32<OutT>(zs.w + c * u.w);
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -276,18 +276,24 @@ __global__ void __launch_bounds__(256, 2)
     for (int i = 0; i < 16; ++i) __stcs(&S4[(warp * 16 + i) * 32 + lane], s[i]);
 }
 
+// out_f32 != 0 writes o in fp32 whatever the input dtype (the layer's use).
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int out_f32) {
     const int nbh = B * H;
     if (nbh == 0) return KDA_OK;
     if (dtype == KDA_BF16) {
-        recurrent_fwd_kernel<__nv_bfloat16><<<nbh, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), g, beta, state, static_cast<__nv_bfloat16*>(o), Tn, H, scale,
-            l2norm);
+        auto qb = static_cast<const __nv_bfloat16*>(q);
+        auto kb = static_cast<const __nv_bfloat16*>(k);
+        auto vb = static_cast<const __nv_bfloat16*>(v);
+        if (out_f32)
+            recurrent_fwd_kernel<__nv_bfloat16, float><<<nbh, 256, 0, stream>>>(
+                qb, kb, vb, g, beta, state, static_cast<float*>(o), Tn, H, scale, l2norm);
+        else
+            recurrent_fwd_kernel<__nv_bfloat16, __nv_bfloat16><<<nbh, 256, 0, stream>>>(
+                qb, kb, vb, g, beta, state, static_cast<__nv_bfloat16*>(o), Tn, H, scale, l2norm);
     } else {
-        recurrent_fwd_kernel<float><<<nbh, 256, 0, stream>>>(
+        recurrent_fwd_kernel<float, float><<<nbh, 256, 0, stream>>>(
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), g, beta, state,
             static_cast<float*>(o), Tn, H, scale, l2norm);
     }

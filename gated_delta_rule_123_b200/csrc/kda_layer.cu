@@ -8,31 +8,28 @@
 // followed by sigmoid, hidden -> 128 -> H*128 alpha gate, FusedRMSNormGated with
 // a sigmoid activation).
 //
-// Pipeline (all on the caller's stream):
-//   z   = x W_in^T                      one bf16 GEMM: [q|k|v|a_down|g_down|b]
+// Pipeline (all on the caller's stream; every step is a kernel of this library):
+//   z, beta = x W_in^T                  tcgen05 GEMM: z = [q|k|v|a_down|g_down|b] in bf16,
+//                                        and beta = sigmoid(b) in fp32 from its epilogue
 //   q,k,v = SiLU(conv4(z_qkv))          causal, restarts at each packed sequence;
-//   q,k <- q,k / ||.||                  fused, one warp per (token, head, tensor)
-//   a   = a_down W_aup^T;  g = -softplus(a) (fp32);  beta = sigmoid(b)
-//   o   = KDA(q, k, v, g, beta)         kda chunk kernels (varlen)
-//   gate = g_down W_gup^T
-//   on  = RMSNorm_head(o) * norm_w * sigmoid(gate)
-//   y   = on W_o^T
-// The four projections are plain GEMMs and run on cuBLASLt; every other step
-// is a kernel of this library.
-#include <cublasLt.h>
-
-#include "kda_common.cuh"
+//   q,k <- q,k / ||.||                  fused into the convolution kernel
+//   g     = -softplus(a_down W_aup^T)   tcgen05 GEMM, fp32 from its epilogue
+//   o     = KDA(q, k, v, g, beta)       the chunk kernels (varlen), o kept in fp32
+//   on    = RMSNorm_head(o) * norm_w * sigmoid(g_down W_gup^T)
+//                                        tcgen05 GEMM with the norm and gate in its epilogue
+//   y     = on W_o^T                    tcgen05 GEMM
+#include "kda_gemm.cuh"
 
 namespace kda {
 
 int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      const float* init, float* fin, void* o, const int32_t* cu, int num_seqs, int B, int T, int H,
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
-                     const char** why, int scalar_gate);
+                     const char** why, int scalar_gate, int out_f32);
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
-                         cudaStream_t stream);
+                         cudaStream_t stream, int out_f32);
 
 // Sequence of token t: packed (cu[n] <= t < cu[n+1]), or dense with seq_len
 // tokens per sequence when cu is NULL.
@@ -175,107 +172,10 @@ __global__ void conv_cache_out_kernel(const __nv_bfloat16* __restrict__ z, int l
     for (int j = 0; j < 3; ++j) conv_out[((size_t)n * 3 + j) * C + c] = r[j];
 }
 
-// g = -softplus(a) (fp32, per channel); beta = sigmoid(b_raw) (per token, head).
-__global__ void gates_kernel(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ z, int ldz,
-                             int off_b, long long ntok, int H, float* __restrict__ g, float* __restrict__ beta) {
-    const long long HD = (long long)H * kD;
-    const long long n4 = ntok * HD / 4;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-        const uint2 raw = reinterpret_cast<const uint2*>(a)[i];
-        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        const float xv[4] = {__low2float(pr[0]), __high2float(pr[0]), __low2float(pr[1]), __high2float(pr[1])};
-        float4 r;
-        float* rr = reinterpret_cast<float*>(&r);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float x = xv[u];
-            rr[u] = -(fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))));
-        }
-        reinterpret_cast<float4*>(g)[i] = r;
-    }
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < ntok * H; i += (long long)gridDim.x * blockDim.x) {
-        const long long t = i / H;
-        const int h = int(i % H);
-        const float x = __bfloat162float(z[t * ldz + off_b + h]);
-        beta[i] = 1.f / (1.f + __expf(-x));
-    }
-}
-
-// on = o / sqrt(mean(o^2) + 1e-5) * norm_w * sigmoid(gate), one warp per (token, head).
-__global__ void norm_gate_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ gate,
-                                 const float* __restrict__ norm_w, long long rows, __nv_bfloat16* __restrict__ out) {
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const uint2 ro = *reinterpret_cast<const uint2*>(o + row * kD + lane * 4);
-    const uint2 rg = *reinterpret_cast<const uint2*>(gate + row * kD + lane * 4);
-    const __nv_bfloat162* po = reinterpret_cast<const __nv_bfloat162*>(&ro);
-    const __nv_bfloat162* pg = reinterpret_cast<const __nv_bfloat162*>(&rg);
-    const float ov[4] = {__low2float(po[0]), __high2float(po[0]), __low2float(po[1]), __high2float(po[1])};
-    const float gv[4] = {__low2float(pg[0]), __high2float(pg[0]), __low2float(pg[1]), __high2float(pg[1])};
-    float ss = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) ss += ov[u] * ov[u];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float rs = rsqrtf(ss * (1.f / kD) + 1e-5f);
-    float r[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) r[u] = ov[u] * rs * norm_w[lane * 4 + u] / (1.f + __expf(-gv[u]));
-    __nv_bfloat162 o2[2] = {__floats2bfloat162_rn(r[0], r[1]), __floats2bfloat162_rn(r[2], r[3])};
-    *reinterpret_cast<uint2*>(out + row * kD + lane * 4) = *reinterpret_cast<uint2*>(o2);
-}
-
-// ---------------------------------------------------------------- cuBLASLt
-static cublasLtHandle_t lt_handle() {
-    static cublasLtHandle_t h = nullptr;
-    if (!h && cublasLtCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
-    return h;
-}
-
-// Row-major C[M,N] = A[M,K] (leading dim lda) * W[N,K]^T, bf16 in/out, fp32 accumulate.
-static bool gemm_bf16(const void* A, int lda, const void* W, int ldw, void* C, int ldc, int M, int N, int K,
-                      void* ws, size_t ws_bytes, cudaStream_t stream) {
-    cublasLtHandle_t h = lt_handle();
-    if (!h) return false;
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-    cublasLtMatmulPreference_t pref = nullptr;
-    bool ok = false;
-    const cublasOperation_t tA = CUBLAS_OP_T, tB = CUBLAS_OP_N;
-    do {
-        if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
-        cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &tA, sizeof(tA));
-        cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tB, sizeof(tB));
-        // column-major view: C^T [N x M] = W [K x N]^T * A^T [K x M]
-        if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, N, ldw) != CUBLAS_STATUS_SUCCESS) break;
-        if (cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, lda) != CUBLAS_STATUS_SUCCESS) break;
-        if (cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, N, M, ldc) != CUBLAS_STATUS_SUCCESS) break;
-        if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
-        cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                             sizeof(ws_bytes));
-        cublasLtMatmulHeuristicResult_t res;
-        int nres = 0;
-        if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &nres) != CUBLAS_STATUS_SUCCESS ||
-            nres == 0)
-            break;
-        const float alpha = 1.f, beta = 0.f;
-        ok = cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, C, lc, C, lc, &res.algo, ws, ws_bytes, stream) ==
-             CUBLAS_STATUS_SUCCESS;
-    } while (0);
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    if (lc) cublasLtMatrixLayoutDestroy(lc);
-    if (lb) cublasLtMatrixLayoutDestroy(lb);
-    if (la) cublasLtMatrixLayoutDestroy(la);
-    if (op) cublasLtMatmulDescDestroy(op);
-    return ok;
-}
-
 struct LayerPlan {
     int HD, nz, ldz;  // ldz: row stride of z, padded to 8 elements so every row is 16-byte aligned
-    size_t off_z, off_q, off_k, off_v, off_a, off_g, off_beta, off_o, off_lt, off_chunk, chunk_bytes, total;
+    size_t off_z, off_q, off_k, off_v, off_g, off_beta, off_o, off_chunk, chunk_bytes, total;
 };
-constexpr size_t kLtWorkspace = 32u << 20;
 
 static size_t up256l(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -288,14 +188,12 @@ static LayerPlan make_layer_plan(int ntok, int d_model, int H, int rank, int nse
     size_t off = 0;
     const size_t tokHD = size_t(ntok) * p.HD;
     p.off_z = off; off = up256l(off + size_t(ntok) * p.ldz * 2);
-    p.off_q = off; off = up256l(off + tokHD * 2);
+    p.off_q = off; off = up256l(off + tokHD * 2);  // q, then the normed and gated output
     p.off_k = off; off = up256l(off + tokHD * 2);
     p.off_v = off; off = up256l(off + tokHD * 2);
-    p.off_a = off; off = up256l(off + tokHD * 2);
     p.off_g = off; off = up256l(off + tokHD * 4);
     p.off_beta = off; off = up256l(off + size_t(ntok) * H * 4);
-    p.off_o = off; off = up256l(off + tokHD * 2);
-    p.off_lt = off; off = up256l(off + kLtWorkspace);
+    p.off_o = off; off = up256l(off + tokHD * 4);  // the operator's output, fp32
     p.chunk_bytes = chunked ? chunk_workspace_bytes(1, ntok, H, nseq, KDA_BF16, 0) : 0;
     p.off_chunk = off; off = up256l(off + p.chunk_bytes);
     p.total = off;
@@ -328,18 +226,18 @@ static int layer_pipeline(const void* x, const kda_layer_weights* w, const int32
     __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(b + pl.off_q);
     __nv_bfloat16* k = reinterpret_cast<__nv_bfloat16*>(b + pl.off_k);
     __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(b + pl.off_v);
-    __nv_bfloat16* a = reinterpret_cast<__nv_bfloat16*>(b + pl.off_a);
     float* g = reinterpret_cast<float*>(b + pl.off_g);
     float* beta = reinterpret_cast<float*>(b + pl.off_beta);
-    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(b + pl.off_o);
-    void* lt = b + pl.off_lt;
+    float* o = reinterpret_cast<float*>(b + pl.off_o);
     const int HD = pl.HD, nz = pl.nz, ldz = pl.ldz;
     const __nv_bfloat16* zb = z;
 
-    if (!gemm_bf16(x, D, w->W_in, D, z, ldz, ntok, nz, D, lt, kLtWorkspace, stream)) {
-        *why = "cuBLASLt input projection failed";
-        return KDA_ERR_CUDA;
-    }
+    GemmEpilogue ep_in;  // z in bf16; the beta columns also as sigmoid in fp32
+    ep_in.beta_out = beta;
+    ep_in.beta_col0 = 3 * HD + 2 * R;
+    ep_in.H = H;
+    int rc = launch_gemm(x, D, w->W_in, D, z, ldz, ntok, nz, D, ep_in, stream, why);
+    if (rc != KDA_OK) return rc;
     {
         const dim3 grid(unsigned((ntok + kConvTok - 1) / kConvTok), 3, unsigned((HD + 2047) / 2048));
         conv_silu_norm_kernel<<<grid, 256, 0, stream>>>(zb, ldz, static_cast<const __nv_bfloat16*>(w->conv_w), cu,
@@ -352,34 +250,30 @@ static int layer_pipeline(const void* x, const kda_layer_weights* w, const int32
             zb, ldz, cu, nseq, seq_len, 3 * HD, static_cast<const __nv_bfloat16*>(conv_in),
             static_cast<__nv_bfloat16*>(conv_out));
     }
-    if (!gemm_bf16(zb + 3 * HD, ldz, w->W_aup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
-        *why = "cuBLASLt alpha up-projection failed";
-        return KDA_ERR_CUDA;
-    }
-    gates_kernel<<<1184, 256, 0, stream>>>(a, zb, ldz, 3 * HD + 2 * R, ntok, H, g, beta);
+    GemmEpilogue ep_decay;  // g = -softplus(a_down W_aup^T), fp32
+    ep_decay.kind = GemmEpilogue::kNegSoftplus;
+    rc = launch_gemm(zb + 3 * HD, ldz, w->W_aup, R, g, HD, ntok, HD, R, ep_decay, stream, why);
+    if (rc != KDA_OK) return rc;
     if (decode) {
-        const int rc = launch_recurrent_fwd(q, k, v, g, beta, state_inplace, o, nseq, seq_len, H, KDA_BF16, 1.f, 0,
-                                            stream);
+        rc = launch_recurrent_fwd(q, k, v, g, beta, state_inplace, o, nseq, seq_len, H, KDA_BF16, 1.f, 0, stream, 1);
         if (rc != KDA_OK) {
             *why = "recurrent kernel launch failed";
             return rc;
         }
     } else {
-        const int rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
-                                        b + pl.off_chunk, pl.chunk_bytes, stream, why, 0);
+        rc = launch_chunk_fwd(q, k, v, g, beta, init, fin, o, cu, nseq, 1, ntok, H, KDA_BF16, 1.f, 0,
+                              b + pl.off_chunk, pl.chunk_bytes, stream, why, 0, 1);
         if (rc != KDA_OK) return rc;
     }
-    // output gate pre-activation reuses the alpha buffer
-    if (!gemm_bf16(zb + 3 * HD + R, ldz, w->W_gup, R, a, HD, ntok, HD, R, lt, kLtWorkspace, stream)) {
-        *why = "cuBLASLt gate up-projection failed";
-        return KDA_ERR_CUDA;
-    }
-    const long long rows = (long long)ntok * H;
-    norm_gate_kernel<<<unsigned((rows + 7) / 8), 256, 0, stream>>>(o, a, w->norm_w, rows, q);
-    if (!gemm_bf16(q, HD, w->W_o, HD, y, D, ntok, D, HD, lt, kLtWorkspace, stream)) {
-        *why = "cuBLASLt output projection failed";
-        return KDA_ERR_CUDA;
-    }
+    GemmEpilogue ep_gate;  // RMSNorm_head(o) * norm_w * sigmoid(g_down W_gup^T), bf16 (over q)
+    ep_gate.kind = GemmEpilogue::kNormGate;
+    ep_gate.o_in = o;
+    ep_gate.ldo = HD;
+    ep_gate.norm_w = w->norm_w;
+    rc = launch_gemm(zb + 3 * HD + R, ldz, w->W_gup, R, q, HD, ntok, HD, R, ep_gate, stream, why);
+    if (rc != KDA_OK) return rc;
+    rc = launch_gemm(q, HD, w->W_o, HD, y, D, ntok, D, HD, GemmEpilogue{}, stream, why);
+    if (rc != KDA_OK) return rc;
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         *why = cudaGetErrorString(e);

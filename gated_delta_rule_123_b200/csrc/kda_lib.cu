@@ -5,5 +5,6 @@
 #include "kda_dplr.cu"
 #include "kda_decode.cu"
 #include "kda_backward.cu"
+#include "kda_gemm.cu"
 #include "kda_layer.cu"
 #include "kda_noalloc.cu"

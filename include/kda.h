@@ -358,9 +358,32 @@ int kda_recurrent_bwd(const void *q, const void *k, const void *v, const float *
  *           conv_state_in.  Together with final_state this is the fixed-size
  *           cache the pages describe ("Training and Inference": KDA caches the
  *           short-convolution state and the recurrent state).
- * Projections run on cuBLASLt (plain bf16 GEMMs, fp32 accumulate); everything
- * else runs in this library's kernels.
+ * Every step runs in this library's kernels: the projections on the tensor
+ * cores (kda_linear_bf16's GEMM, bf16 operands, fp32 accumulation), with beta,
+ * the log decay g = -softplus(.) and the RMSNorm x sigmoid(gate) computed in
+ * the epilogues of the GEMMs that produce their inputs; the operator's output
+ * o stays fp32 up to the RMSNorm.  Intermediate activations (the projections,
+ * q, k, v after the convolution, the normed output) are bf16.
  */
+/* ------------------------------------------------------------------------
+ * kda_linear_bf16 -- one projection of the KDA layer: y = x W^T.
+ *
+ * "Kimi Linear: An Expressive, Efficient Attention Architecture", section
+ * "Neural Parameterization": the layer's Q/K/V, gate and output projections
+ * are bias-free linear maps.  kda_layer_fwd runs all of them on this GEMM
+ * (tcgen05 tensor cores, TMA-fed, fp32 accumulation in tensor memory); this
+ * entry point exposes the plain form.
+ *
+ *   x   bf16 [M, K] row-major, row stride ldx elements;
+ *   W   bf16 [N, K] row-major ("out x in"), row stride ldw;
+ *   y   bf16 [M, N] row-major, row stride ldy; rounded from the fp32
+ *       accumulator to nearest, ties to even.  Must not alias x or W.
+ * Pointers 16-byte aligned and row strides multiples of 8 elements.  Any
+ * M, N, K >= 1.  No workspace.
+ */
+int kda_linear_bf16(const void *x, int ldx, const void *W, int ldw, void *y, int ldy, int M, int N, int K,
+                    void *stream);
+
 typedef struct {
     const void *W_in;
     const void *W_aup;
