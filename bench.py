@@ -223,6 +223,63 @@ def time_layer(kda, synth, dev, rank, time_calls, tc_peak, world):
             "frac": flop / (ms / 1e3) / 1e12 / tc_peak, "gemm": gemms}
 
 
+DPLR_BYTES_PER_TOKEN_HEAD = 5 * D * 2 + D * 2 + D * 4 + 4  # q,k,v,a,b + o (bf16), g (fp32), beta
+
+
+def time_sweep(kda, synth, dev, rank, time_calls, hbm_peak, world, ms_64k, gdn_ms_64k):
+    """The pages' length sweep (B=1, H=16, T = 8K..64K) for KDA, its scalar-gate special case
+    (gated DeltaNet) and the untied DPLR kernel, each as tokens/s and as the fraction of HBM
+    bandwidth its algorithmic bytes reach; plus KDA against DPLR at T=65536 with neither
+    kernel running the segment scan (B=4, H=16: 64 CTAs, one per sequence and head)."""
+    import torch
+    rows = []
+    for T in synth.PREFILL_SWEEP_T:
+        cfg = dict(synth.prefill_sweep(T))
+        cfg["seed"] += 1000 * rank
+        row = {"T": T}
+        if T == T_PREFILL and ms_64k is not None:
+            kms, gms = ms_64k, gdn_ms_64k
+        else:
+            inp = synth.op_inputs(**cfg, device=dev)
+            o, fs = torch.empty_like(inp["q"]), torch.empty_like(inp["s0"])
+            ws = torch.empty(kda.chunk_fwd_workspace_bytes(1, T, H_PREFILL), device=dev, dtype=torch.uint8)
+            args5 = [inp[n] for n in ("q", "k", "v", "g", "beta")]
+            kms = time_calls(lambda: kda.chunk_fwd(*args5, initial_state=inp["s0"], out=o, final_state=fs,
+                                                   workspace=ws), 10)
+            gs = inp["g"][..., 0].contiguous()
+            gms = time_calls(lambda: kda.gdn_chunk_fwd(args5[0], args5[1], args5[2], gs, args5[4],
+                                                       initial_state=inp["s0"], out=o, final_state=fs,
+                                                       workspace=ws), 10)
+            del inp, o, fs, ws, args5, gs
+        dp = synth.dplr_inputs(**cfg, device=dev)
+        do, dfs = torch.empty_like(dp["q"]), torch.empty_like(dp["s0"])
+        dargs = [dp[n] for n in ("q", "k", "v", "a", "b", "g", "beta")]
+        dms = time_calls(lambda: kda.dplr_chunk_fwd(*dargs, initial_state=dp["s0"], out=do, final_state=dfs), 3)
+        del dp, do, dfs, dargs
+        for name, ms, bpt in (("kda", kms, BYTES_PER_TOKEN_HEAD), ("gdn", gms, GDN_BYTES_PER_TOKEN_HEAD),
+                              ("dplr", dms, DPLR_BYTES_PER_TOKEN_HEAD)):
+            gbs = bpt * T * H_PREFILL / (ms / 1e3) / 1e9
+            row[name] = {"ms": ms, "tokens_per_s": world * T / (ms / 1e3), "hbm_frac": gbs / hbm_peak}
+        rows.append(row)
+    # like for like at the pages' comparison length: 64 (sequence, head) pairs, one CTA each
+    B4, T4 = 4, T_PREFILL
+    dp = synth.dplr_inputs(B=B4, H=H_PREFILL, T=T4, s0_std=0.02, seed=31 + rank, device=dev)
+    do, dfs = torch.empty_like(dp["q"]), torch.empty_like(dp["s0"])
+    assert kda.chunk_fwd_segments(B4, T4, H_PREFILL) == (0, 0)
+    ws = torch.empty(kda.chunk_fwd_workspace_bytes(B4, T4, H_PREFILL), device=dev, dtype=torch.uint8)
+    kms = time_calls(lambda: kda.chunk_fwd(*(dp[n] for n in ("q", "k", "v", "g", "beta")), initial_state=dp["s0"],
+                                           out=do, final_state=dfs, workspace=ws), 3)
+    dms = time_calls(lambda: kda.dplr_chunk_fwd(*(dp[n] for n in ("q", "k", "v", "a", "b", "g", "beta")),
+                                                initial_state=dp["s0"], out=do, final_state=dfs), 3)
+    del dp, do, dfs, ws
+    return {"workload": "B=1 H=16 d=128, T = 8K..64K (prefill distributions); kda = per-channel gates, "
+                        "gdn = one gate per token-head, dplr = untied a, b",
+            "lengths": rows,
+            "no_scan_64k": {"workload": f"B={B4} H=16 T={T4}: 64 CTAs, one per (sequence, head); neither "
+                                        "kernel segments", "kda_ms": kms, "dplr_ms": dms,
+                            "dplr_over_kda": dms / kms}}
+
+
 def run_ours(args):
     import torch
 
@@ -266,6 +323,31 @@ def run_ours(args):
         torch.cuda.synchronize()
         return max_over_ranks(start.elapsed_time(end) / n)
 
+    if args.gemm_only:  # the layer's input projection shape with args.gemm_m rows (profiling runs)
+        lc = synth.LAYER_65K
+        n_out = 3 * lc["H"] * D + 2 * lc["rank"] + lc["H"]
+        gen = torch.Generator(device=dev).manual_seed(9)
+        a = torch.randn((args.gemm_m, lc["d_model"]), device=dev, generator=gen).to(torch.bfloat16)
+        w = (0.02 * torch.randn((n_out, lc["d_model"]), device=dev, generator=gen)).to(torch.bfloat16)
+        yo = torch.empty((args.gemm_m, n_out), device=dev, dtype=torch.bfloat16)
+        gms = time_calls(lambda: kda.linear(a, w, out=yo), args.steps)
+        tf = 2 * args.gemm_m * n_out * lc["d_model"] / (gms / 1e3) / 1e12
+        if rank == 0:
+            print(json.dumps({"metric": "GEMM TFLOP/s", "value": tf, "unit": "TFLOP/s", "ms": gms,
+                              "config": {"workload": f"y = x W^T, M={args.gemm_m} N={n_out} K={lc['d_model']} bf16"},
+                              "frac": tf / tc_peak}), flush=True)
+        ranks.close()
+        return 0
+    if args.dplr_only:  # the untied DPLR kernel at B=1, H=16, T=args.T (profiling runs)
+        dp = synth.dplr_inputs(**synth.prefill_sweep(T), device=dev)
+        do, dfs = torch.empty_like(dp["q"]), torch.empty_like(dp["s0"])
+        dms = time_calls(lambda: kda.dplr_chunk_fwd(*(dp[n] for n in ("q", "k", "v", "a", "b", "g", "beta")),
+                                                    initial_state=dp["s0"], out=do, final_state=dfs), args.steps)
+        if rank == 0:
+            print(json.dumps({"metric": "DPLR prefill tokens/s", "value": T / (dms / 1e3), "unit": "tokens/s",
+                              "ms": dms, "config": {"workload": f"untied DPLR B=1 H=16 T={T}"}}), flush=True)
+        ranks.close()
+        return 0
     if args.layer_only:
         layer = time_layer(kda, synth, dev, rank, time_calls, tc_peak, world)
         if rank == 0:
@@ -465,6 +547,9 @@ def run_ours(args):
 
     layer = time_layer(kda, synth, dev, rank, time_calls, tc_peak, world)
     assert kda.device_status() == 0
+    sweep = time_sweep(kda, synth, dev, rank, time_calls, hbm_peak, world, ms if T == T_PREFILL else None,
+                       gdn_ms if T == T_PREFILL else None)
+    assert kda.device_status() == 0
 
     # End to end through the public call with host buffers (pinned), copies inside the timed
     # region.  Steps are pipelined as a serving loop would run them: step i+1's inputs go
@@ -558,6 +643,7 @@ def run_ours(args):
             "backward": {"workload": "B=1 H=16 T=8192: dq, dk, dv, dg, dbeta, dS0 by recurrent reverse mode",
                          "ms_per_call": bwd_ms, "tokens_per_s": world * bT / (bwd_ms / 1e3)},
             "layer": layer,
+            "sweep": sweep,
             "gdn": {"workload": f"gated DeltaNet prefill B=1 H=16 T={T}, one fp32 log-gate per token-head",
                     "ms_per_step": gdn_ms, "tokens_per_s": world * T / (gdn_ms / 1e3),
                     "step_gbs": gdn_bytes / (gdn_ms / 1e3) / 1e9,
@@ -579,6 +665,9 @@ def main():
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and the CPU baseline")
     ap.add_argument("--eager", action="store_true", help="time the prefill calls as issued, not as one CUDA graph")
     ap.add_argument("--layer-only", action="store_true", help="time only the KDA layer (profiling runs)")
+    ap.add_argument("--gemm-only", action="store_true", help="time only the layer's input-projection GEMM")
+    ap.add_argument("--gemm-m", type=int, default=65536, help="rows of the --gemm-only GEMM")
+    ap.add_argument("--dplr-only", action="store_true", help="time only the untied DPLR kernel at --T")
     ap.add_argument("--warmup-seconds", type=float, default=1.5, help="minimum warm-up time (clock sampling)")
     args = ap.parse_args()
     if args.warmup < 3:

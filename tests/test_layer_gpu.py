@@ -59,11 +59,12 @@ def test_layer_many_short_sequences_no_state(kda):
 @pytest.mark.slow
 def test_layer_full_size_sampled_sequences(kda):
     """d_model=2048, H=16, 65536 packed tokens in 8 sequences (rank 128): the
-    oracle checks the two shortest sequences end to end."""
+    oracle checks the two shortest sequences and the longest one (whose 191
+    chunks bound the operator's launch) end to end."""
     cfg = synth.LAYER_65K
     cu = synth.random_cu_seqlens(cfg["Ttot"], cfg["nseq"], cfg["seed"])
     lens = np.diff(cu)
-    pick = list(np.argsort(lens)[:2])
+    pick = list(np.argsort(lens)[:2]) + [int(np.argmax(lens))]
     errs = run_layer(kda, d_model=cfg["d_model"], H=cfg["H"], Ttot=cfg["Ttot"], nseq=cfg["nseq"], rank=cfg["rank"],
                      seed=cfg["seed"], check_seqs=pick)
     for ey, es in errs:
