@@ -13,24 +13,63 @@
 // chunk form, with FLA's tests covering q/k/v/g/beta and initial-state
 // gradients); this kernel computes them exactly (fp32) by recurrence.
 //
-// Layout: one CTA (256 threads) per (sequence, head); warp w owns key rows
-// [16w, 16w+16), lane l value columns [4l, 4l+4); S, G and S~ live in
-// registers.  Phase 1 runs the forward and stores the state at every 64-token
-// boundary (checkpoints in the workspace).  Phase 2 walks the chunks backwards:
-// it recomputes the chunk's 64 intermediate states from its checkpoint into a
-// per-CTA scratch (4 MB, L2-resident), then runs the reverse steps reading them
-// back.  Column sums (y, du) go through shared memory, one barrier each; row sums
-// (dq, dk, dg) are butterfly reductions over the 32 lanes: 16 partial row sums
-// per lane become one full sum per lane pair in 16 shuffles.
+// Parallel layout.  The recurrence never mixes value columns: column j of S and
+// of G evolves on its own (y, u, du and dy are per-column).  So every (sequence,
+// head) is split into kSlices = 16 CTAs of kSliceCols = 8 value columns each
+// (small enough that two CTAs share an SM), and a CTA
+// runs the whole sequence for its columns with one key row per thread (128
+// threads): the per-column sums y = S~^T k and du = G^T k are a warp
+// reduce-scatter plus one barrier per token, and the per-row sums dq, dk, dg (and
+// the scalar dbeta) are in-thread partial sums over the CTA's columns.  Those
+// partials go to the workspace and a second kernel adds the slices up (in a fixed
+// order, so results are deterministic); dv and the initial-state gradient are
+// per-column and written directly.
+//   Phase 1 runs the forward and stores the state slice at every kSub-token
+//   boundary.  Phase 2 walks the sub-chunks backwards: it recomputes the kSub
+//   states S_{t-1} of a sub-chunk from its checkpoint into shared memory, then
+//   runs the reverse steps reading them back.  Each sub-chunk's token inputs (k,
+//   q, g per row; the slice's v and dO; beta) are staged into shared memory with
+//   cp.async one sub-chunk ahead, so a step reads nothing from global memory.
 #include "kda_common.cuh"
 
 namespace kda {
+namespace bwd {
 
-// Sum x[i] (i < 16, the 16 rows of this warp) over the 32 lanes.  Returns the
-// full sum of row (lane >> 1) & 15 (each lane pair holds the same row).
-__device__ __forceinline__ float rowsum_16x32(float (&x)[16], int lane) {
+constexpr int kSliceCols = 8;                  // value columns per CTA
+constexpr int kSlices = kD / kSliceCols;       // CTAs per (sequence, head)
+constexpr int kSub = 16;                       // tokens per recomputed / staged sub-chunk
+constexpr int kThreads = kD;                   // one key row per thread
+constexpr uint32_t kStateBytes = kSub * kSliceCols * kD * sizeof(float);  // states [kSub][col][row]
+
+// One sub-chunk of token inputs in shared memory (element type E of q, k, v, dO):
+// k, q [kSub][128]; g fp32 [kSub][128]; the slice's v, dO [kSub][16]; beta [kSub].
+template <typename E>
+struct Stage {
+    static constexpr uint32_t K = 0, Q = kSub * kD * sizeof(E), G = 2 * Q, V = G + kSub * kD * 4,
+                              DO = V + kSub * kSliceCols * sizeof(E), B = DO + kSub * kSliceCols * sizeof(E),
+                              kBytes = (B + kSub * 4 + 127) & ~127u;
+};
+template <typename E>
+constexpr uint32_t smem_bytes() { return kStateBytes + 2 * Stage<E>::kBytes; }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Sum x[c] (c < N) over the 32 lanes of the warp.  Returns, in every lane, the full
+// sum of column lane / (32 / N) (groups of 32 / N lanes hold the same column): a
+// reduce-scatter that halves the values per lane at each step, then plain sums.
+template <int N>
+__device__ __forceinline__ float colsum_x32(float (&x)[N], int lane) {
+    int off = 16;
 #pragma unroll
-    for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
+    for (int half = N / 2; half >= 1; half >>= 1, off >>= 1) {
         const bool hi = (lane & off) != 0;
 #pragma unroll
         for (int j = 0; j < half; ++j) {
@@ -39,225 +78,311 @@ __device__ __forceinline__ float rowsum_16x32(float (&x)[16], int lane) {
             x[j] = (hi ? x[j + half] : x[j]) + recv;
         }
     }
-    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+    float sum = x[0];
+#pragma unroll
+    for (; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    return sum;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreads)
     recurrent_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                          const float* __restrict__ g, const float* __restrict__ beta, const float* __restrict__ init,
-                         const T* __restrict__ dout, const float* __restrict__ dfinal, float* __restrict__ dq,
-                         float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg,
-                         float* __restrict__ dbeta, float* __restrict__ dinit, float4* __restrict__ ckpt,
-                         float4* __restrict__ scratch, int Tn, int H, float scale) {
-    __shared__ __align__(16) float sk[2][kD], sq[2][kD], sa[2][kD], sv[2][kD], sdo[2][kD];
-    __shared__ float sb[2];
-    __shared__ float4 sy[2][8][32], sdu[2][8][32];
+                         const T* __restrict__ dout, const float* __restrict__ dfinal, float* __restrict__ dv,
+                         float* __restrict__ dinit, float* __restrict__ part, float* __restrict__ ckpt, int Tn, int H,
+                         float scale) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* sst = reinterpret_cast<float*>(smem);  // [kSub][kSliceCols][kD]: S_{t-1} of the sub-chunk's tokens
+    __shared__ __align__(16) float red[2][4][2][kSliceCols];  // per parity, warp: y and du partials
+    using S = Stage<T>;
 
-    const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nchunks = (Tn + kC - 1) / kC;
+    const int bh = blockIdx.x, sl = blockIdx.y, b = bh / H, h = bh - b * H;
+    const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+    const int c0 = sl * kSliceCols;
+    const int nsub = (Tn + kSub - 1) / kSub;
+    const size_t TH = size_t(gridDim.x) * Tn;  // (sequence, token, head) rows: [B][Tn][H]
     auto row = [&](int t) { return (size_t(b) * Tn + t) * H + h; };
-    auto sidx4 = [&](int i) { return (warp * 16 + i) * 32 + lane; };  // float4 index of (row 16w+i, cols 4l..)
-    float4* ck = ckpt + size_t(bh) * nchunks * (kD * kD / 4);
-    float4* sc = scratch + size_t(bh) * kC * (kD * kD / 4);
+    // per-slice partial sums: [slice][dq | dk | dg][B*Tn*H][kD], then dbeta [slice][B*Tn*H]
+    float* p_dq = part + (size_t(sl) * 3 + 0) * TH * kD;
+    float* p_dk = part + (size_t(sl) * 3 + 1) * TH * kD;
+    float* p_dg = part + (size_t(sl) * 3 + 2) * TH * kD;
+    float* p_db = part + size_t(kSlices) * 3 * TH * kD + size_t(sl) * TH;
+    float* ck = ckpt + (size_t(bh) * kSlices + sl) * size_t(nsub) * (kSliceCols * kD);  // [nsub][col][row]
+    const uint32_t stage0 = smem_u32(smem + kStateBytes);
 
-    // token vectors into buffer p (threads < 128: one channel each); q is pre-scaled
-    auto load_tok = [&](int t, int p, bool with_bwd) {
-        if (tid < kD) {
-            const size_t e = row(t) * kD + tid;
-            sk[p][tid] = to_f32(k[e]);
-            sa[p][tid] = expf(g[e]);
-            sv[p][tid] = to_f32(v[e]);
-            if (with_bwd) {
-                sq[p][tid] = to_f32(q[e]) * scale;
-                sdo[p][tid] = to_f32(dout[e]);
+    // Stage sub-chunk sc into buffer buf with cp.async (every thread issues its share;
+    // tokens past the end read as zero).  One commit group per call.
+    auto stage = [&](int sc, int buf, bool with_bwd) {
+        const uint32_t base = stage0 + uint32_t(buf) * S::kBytes;
+        constexpr int per_row = kD * sizeof(T) / 16;           // 16-byte pieces of a 128-wide row
+        constexpr int per_slice = kSliceCols * sizeof(T) / 16;  // of the slice's 16 values
+        for (int i = r; i < kSub * per_row; i += kThreads) {
+            const int j = i / per_row, piece = i % per_row, t = sc * kSub + j;
+            const bool ok = t < Tn;
+            const size_t e = (ok ? row(t) : 0) * kD;
+            const uint32_t off = uint32_t(j * kD * sizeof(T) + piece * 16);
+            cp_async16(base + S::K + off, reinterpret_cast<const uint8_t*>(k + e) + piece * 16, ok ? 16u : 0u);
+            if (with_bwd)
+                cp_async16(base + S::Q + off, reinterpret_cast<const uint8_t*>(q + e) + piece * 16, ok ? 16u : 0u);
+        }
+        for (int i = r; i < kSub * (kD * 4 / 16); i += kThreads) {
+            const int j = i / (kD * 4 / 16), piece = i % (kD * 4 / 16), t = sc * kSub + j;
+            const bool ok = t < Tn;
+            const size_t e = (ok ? row(t) : 0) * kD;
+            cp_async16(base + S::G + uint32_t(j * kD * 4 + piece * 16),
+                       reinterpret_cast<const uint8_t*>(g + e) + piece * 16, ok ? 16u : 0u);
+        }
+        if (r < kSub * per_slice) {
+            const int j = r / per_slice, piece = r % per_slice, t = sc * kSub + j;
+            const bool ok = t < Tn;
+            const size_t e = (ok ? row(t) : 0) * kD + c0;
+            const uint32_t off = uint32_t(j * kSliceCols * sizeof(T) + piece * 16);
+            cp_async16(base + S::V + off, reinterpret_cast<const uint8_t*>(v + e) + piece * 16, ok ? 16u : 0u);
+            if (with_bwd)
+                cp_async16(base + S::DO + off, reinterpret_cast<const uint8_t*>(dout + e) + piece * 16,
+                           ok ? 16u : 0u);
+        }
+        if (r < kSub) {
+            const int t = sc * kSub + r;
+            const bool ok = t < Tn;
+            cp_async_4(base + S::B + r * 4, beta + (ok ? row(t) : 0), ok ? 4u : 0u);
+        }
+        cp_commit();
+    };
+    auto sbuf = [&](int buf) { return smem + kStateBytes + buf * S::kBytes; };
+    auto ld = [&](const uint8_t* p) { return to_f32(*reinterpret_cast<const T*>(p)); };
+
+    auto reduce_cols = [&](float (&x)[kSliceCols], int par, int which) {
+        constexpr int kGroup = 32 / kSliceCols;  // lanes holding one column's sum
+        const float s = colsum_x32<kSliceCols>(x, lane);
+        if (lane % kGroup == 0) red[par][warp][which][lane / kGroup] = s;
+    };
+    auto read_cols = [&](float (&out)[kSliceCols], int par, int which) {
+#pragma unroll
+        for (int c4 = 0; c4 < kSliceCols; c4 += 4) {
+            float4 acc = *reinterpret_cast<const float4*>(&red[par][0][which][c4]);
+#pragma unroll
+            for (int w = 1; w < 4; ++w) {
+                const float4 t4 = *reinterpret_cast<const float4*>(&red[par][w][which][c4]);
+                acc.x += t4.x; acc.y += t4.y; acc.z += t4.z; acc.w += t4.w;
             }
-            if (tid == 0) sb[p] = beta[row(t)];
+            out[c4] = acc.x; out[c4 + 1] = acc.y; out[c4 + 2] = acc.z; out[c4 + 3] = acc.w;
         }
     };
-    // one forward step on s with the token in buffer p (two barriers: vectors, partials)
-    auto fwd_step = [&](float4 (&s)[16], int p) {
+    // one forward step of this thread's row of the slice, token j of staged buffer sb (one barrier)
+    auto fwd_step = [&](float (&s)[kSliceCols], const uint8_t* sb, int j, int par) {
+        const float kr = ld(sb + S::K + (j * kD + r) * sizeof(T));
+        const float a = expf(reinterpret_cast<const float*>(sb + S::G)[j * kD + r]);
+        float yp[kSliceCols];
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c) {
+            s[c] *= a;
+            yp[c] = s[c] * kr;
+        }
+        reduce_cols(yp, par, 0);
         __syncthreads();
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        float y[kSliceCols];
+        read_cols(y, par, 0);
+        const float bt = reinterpret_cast<const float*>(sb + S::B)[j];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = warp * 16 + i;
-            const float a = sa[p][r], kr = sk[p][r];
-            s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-            y.x += s[i].x * kr; y.y += s[i].y * kr; y.z += s[i].z * kr; y.w += s[i].w * kr;
-        }
-        sy[p][warp][lane] = y;
-        __syncthreads();
-        float4 ys = sy[p][0][lane];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) {
-            const float4 t4 = sy[p][w][lane];
-            ys.x += t4.x; ys.y += t4.y; ys.z += t4.z; ys.w += t4.w;
-        }
-        const float bt = sb[p];
-        const float4 v4 = reinterpret_cast<const float4*>(sv[p])[lane];
-        const float4 u = make_float4(bt * (v4.x - ys.x), bt * (v4.y - ys.y), bt * (v4.z - ys.z), bt * (v4.w - ys.w));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float kr = sk[p][warp * 16 + i];
-            s[i].x += kr * u.x; s[i].y += kr * u.y; s[i].z += kr * u.z; s[i].w += kr * u.w;
-        }
+        for (int c = 0; c < kSliceCols; ++c)
+            s[c] = fmaf(kr, bt * (ld(sb + S::V + (j * kSliceCols + c) * sizeof(T)) - y[c]), s[c]);
     };
 
-    // ---- phase 1: forward, checkpoint at every chunk start
-    float4 s[16];
-    {
-        const float4* s0 = init ? reinterpret_cast<const float4*>(init) + size_t(bh) * (kD * kD / 4) : nullptr;
+    // ---- phase 1: forward, checkpoint at every sub-chunk start
+    float s[kSliceCols];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) s[i] = s0 ? s0[sidx4(i)] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int c = 0; c < kSliceCols; ++c)
+        s[c] = init ? init[(size_t(bh) * kD + r) * kD + c0 + c] : 0.f;
+    int par = 0;  // parity of the reduction buffer of the next barrier step
+    stage(0, 0, false);
 #pragma unroll 1
-    for (int t = 0; t < Tn; ++t) {
-        if ((t & (kC - 1)) == 0) {
-            float4* dst = ck + size_t(t / kC) * (kD * kD / 4);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) dst[sidx4(i)] = s[i];
+    for (int sc = 0; sc < nsub; ++sc) {
+        if (sc + 1 < nsub) {
+            stage(sc + 1, (sc + 1) & 1, false);
+            cp_wait_1();
+        } else {
+            cp_wait_0();
         }
-        load_tok(t, t & 1, false);
-        fwd_step(s, t & 1);
+        __syncthreads();  // sub-chunk sc has landed for every thread
+        float* dst = ck + size_t(sc) * (kSliceCols * kD);
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c) dst[c * kD + r] = s[c];
+        const uint8_t* sb = sbuf(sc & 1);
+        const int len = min(kSub, Tn - sc * kSub);
+#pragma unroll 1
+        for (int j = 0; j < len; ++j) {
+            fwd_step(s, sb, j, par);
+            par ^= 1;
+        }
+        __syncthreads();  // every thread is done with buffer sc & 1 before it is restaged
     }
 
-    // ---- phase 2: chunks in reverse; G is the running gradient of the state
-    float4 G[16];
-    {
-        const float4* d0 = dfinal ? reinterpret_cast<const float4*>(dfinal) + size_t(bh) * (kD * kD / 4) : nullptr;
+    // ---- phase 2: sub-chunks in reverse; G is the running gradient of the state
+    float G[kSliceCols];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) G[i] = d0 ? d0[sidx4(i)] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int c = 0; c < kSliceCols; ++c)
+        G[c] = dfinal ? dfinal[(size_t(bh) * kD + r) * kD + c0 + c] : 0.f;
+    stage(nsub - 1, (nsub - 1) & 1, true);
 #pragma unroll 1
-    for (int c = nchunks - 1; c >= 0; --c) {
-        const int t0 = c * kC, t1 = min(Tn, t0 + kC);
-        __syncthreads();  // the previous token's readers of the vector buffers are done
-        {  // recompute S_{t-1} for every token of the chunk into the scratch
-            const float4* src = ck + size_t(c) * (kD * kD / 4);
+    for (int sc = nsub - 1; sc >= 0; --sc) {
+        if (sc > 0) {
+            stage(sc - 1, (sc - 1) & 1, true);
+            cp_wait_1();
+        } else {
+            cp_wait_0();
+        }
+        __syncthreads();  // sub-chunk sc has landed for every thread
+        const uint8_t* sb = sbuf(sc & 1);
+        const int t0 = sc * kSub, len = min(kSub, Tn - t0);
+        {  // recompute S_{t-1} of every token of the sub-chunk into shared memory (own row only)
+            const float* src = ck + size_t(sc) * (kSliceCols * kD);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) s[i] = src[sidx4(i)];
+            for (int c = 0; c < kSliceCols; ++c) s[c] = src[c * kD + r];
 #pragma unroll 1
-            for (int t = t0; t < t1; ++t) {
-                float4* dst = sc + size_t(t - t0) * (kD * kD / 4);
+            for (int j = 0; j < len; ++j) {
+                float* dst = sst + j * (kSliceCols * kD);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) dst[sidx4(i)] = s[i];
-                load_tok(t, t & 1, false);
-                fwd_step(s, t & 1);
+                for (int c = 0; c < kSliceCols; ++c) dst[c * kD + r] = s[c];
+                fwd_step(s, sb, j, par);
+                par ^= 1;
             }
         }
-        __syncthreads();  // as above, before the reverse loop reuses the buffers (each thread reads back only its own scratch)
 #pragma unroll 1
-        for (int t = t1 - 1; t >= t0; --t) {
-            const int p = t & 1;
-            float4 St[16];
-            const float4* src = sc + size_t(t - t0) * (kD * kD / 4);
+        for (int j = len - 1; j >= 0; --j) {
+            const int t = t0 + j;
+            const float kr = ld(sb + S::K + (j * kD + r) * sizeof(T));
+            const float qr = ld(sb + S::Q + (j * kD + r) * sizeof(T)) * scale;
+            const float a = expf(reinterpret_cast<const float*>(sb + S::G)[j * kD + r]);
+            const float bt = reinterpret_cast<const float*>(sb + S::B)[j];
+            float d[kSliceCols];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) St[i] = src[sidx4(i)];
-            load_tok(t, p, true);
+            for (int c = 0; c < kSliceCols; ++c) d[c] = ld(sb + S::DO + (j * kSliceCols + c) * sizeof(T));
+            const float* src = sst + j * (kSliceCols * kD);
+            float St[kSliceCols], yp[kSliceCols], dup[kSliceCols];
+#pragma unroll
+            for (int c = 0; c < kSliceCols; ++c) {
+                St[c] = src[c * kD + r] * a;  // S~ = Diag(a) S_{t-1}
+                G[c] = fmaf(qr, d[c], G[c]);
+                yp[c] = St[c] * kr;
+                dup[c] = G[c] * kr;
+            }
+            reduce_cols(yp, par, 0);
+            reduce_cols(dup, par, 1);
             __syncthreads();
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f), du = y;
-            const float4 do4 = reinterpret_cast<const float4*>(sdo[p])[lane];
+            float y[kSliceCols], du[kSliceCols];
+            read_cols(y, par, 0);
+            read_cols(du, par, 1);
+            par ^= 1;
+            float udo = 0.f, dbt = 0.f, xq = 0.f, xk = 0.f, xg = 0.f, dur = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = warp * 16 + i;
-                const float a = sa[p][r], kr = sk[p][r], qr = sq[p][r];
-                St[i].x *= a; St[i].y *= a; St[i].z *= a; St[i].w *= a;  // S~ = Diag(a) S_{t-1}
-                y.x += St[i].x * kr; y.y += St[i].y * kr; y.z += St[i].z * kr; y.w += St[i].w * kr;
-                G[i].x += qr * do4.x; G[i].y += qr * do4.y; G[i].z += qr * do4.z; G[i].w += qr * do4.w;
-                du.x += G[i].x * kr; du.y += G[i].y * kr; du.z += G[i].z * kr; du.w += G[i].w * kr;
+            for (int c = 0; c < kSliceCols; ++c) {
+                const float rr = ld(sb + S::V + (j * kSliceCols + c) * sizeof(T)) - y[c];  // v - y
+                const float u = bt * rr, dy = -bt * du[c];
+                udo = fmaf(u, d[c], udo);
+                dbt = fmaf(du[c], rr, dbt);
+                xq = fmaf(St[c], d[c], xq);
+                xk = fmaf(G[c], u, fmaf(St[c], dy, xk));
+                const float gt = fmaf(kr, dy, G[c]);  // G~ = G + k dy^T
+                xg = fmaf(gt, St[c], xg);
+                G[c] = gt * a;  // G <- Diag(a) G~
+                dur = (c == r) ? du[c] : dur;
             }
-            sy[p][warp][lane] = y;
-            sdu[p][warp][lane] = du;
-            __syncthreads();
-            float4 ys = sy[p][0][lane], dus = sdu[p][0][lane];
-#pragma unroll
-            for (int w = 1; w < 8; ++w) {
-                const float4 a4 = sy[p][w][lane], b4 = sdu[p][w][lane];
-                ys.x += a4.x; ys.y += a4.y; ys.z += a4.z; ys.w += a4.w;
-                dus.x += b4.x; dus.y += b4.y; dus.z += b4.z; dus.w += b4.w;
-            }
-            const float bt = sb[p];
-            const float4 v4 = reinterpret_cast<const float4*>(sv[p])[lane];
-            const float4 r4 = make_float4(v4.x - ys.x, v4.y - ys.y, v4.z - ys.z, v4.w - ys.w);  // v - y
-            const float4 u = make_float4(bt * r4.x, bt * r4.y, bt * r4.z, bt * r4.w);
-            const float4 dy = make_float4(-bt * dus.x, -bt * dus.y, -bt * dus.z, -bt * dus.w);
-            float udo = u.x * do4.x + u.y * do4.y + u.z * do4.z + u.w * do4.w;
-            float dbt = dus.x * r4.x + dus.y * r4.y + dus.z * r4.z + dus.w * r4.w;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                udo += __shfl_xor_sync(0xffffffffu, udo, off);
-                dbt += __shfl_xor_sync(0xffffffffu, dbt, off);
-            }
-            if (warp == 0) {
-                *reinterpret_cast<float4*>(dv + row(t) * kD + 4 * lane) =
-                    make_float4(bt * dus.x, bt * dus.y, bt * dus.z, bt * dus.w);
-                if (lane == 0) dbeta[row(t)] = dbt;
-            }
-            const int rr = warp * 16 + ((lane >> 1) & 15);  // the row this lane pair reduces
-            const bool writer = (lane & 1) == 0;
-            float x[16];
-            // dq = scale (S~ do + k (u . do))
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = St[i].x * do4.x + St[i].y * do4.y + St[i].z * do4.z + St[i].w * do4.w;
-            float sum = rowsum_16x32(x, lane);
-            if (writer) dq[row(t) * kD + rr] = scale * (sum + sk[p][rr] * udo);
-            // dk = G u + S~ dy
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                x[i] = G[i].x * u.x + G[i].y * u.y + G[i].z * u.z + G[i].w * u.w + St[i].x * dy.x + St[i].y * dy.y +
-                       St[i].z * dy.z + St[i].w * dy.w;
-            sum = rowsum_16x32(x, lane);
-            if (writer) dk[row(t) * kD + rr] = sum;
-            // G~ = G + k dy^T;  dg = rowsum(G~ (.) S~);  G <- Diag(a) G~
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = warp * 16 + i;
-                const float kr = sk[p][r], a = sa[p][r];
-                G[i].x += kr * dy.x; G[i].y += kr * dy.y; G[i].z += kr * dy.z; G[i].w += kr * dy.w;
-                x[i] = G[i].x * St[i].x + G[i].y * St[i].y + G[i].z * St[i].z + G[i].w * St[i].w;
-                G[i].x *= a; G[i].y *= a; G[i].z *= a; G[i].w *= a;
-            }
-            sum = rowsum_16x32(x, lane);
-            if (writer) dg[row(t) * kD + rr] = sum;
+            const size_t e = row(t);
+            if (r < kSliceCols) dv[e * kD + c0 + r] = bt * dur;  // dv = beta du: thread r < kSliceCols writes column c0 + r
+            if (r == 0) p_db[e] = dbt;
+            p_dq[e * kD + r] = scale * (xq + kr * udo);
+            p_dk[e * kD + r] = xk;
+            p_dg[e * kD + r] = xg;
         }
+        __syncthreads();  // every thread is done with buffer sc & 1 before it is restaged
     }
     if (dinit) {
-        float4* d = reinterpret_cast<float4*>(dinit) + size_t(bh) * (kD * kD / 4);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) d[sidx4(i)] = G[i];
+        for (int c = 0; c < kSliceCols; ++c) dinit[(size_t(bh) * kD + r) * kD + c0 + c] = G[c];
     }
 }
 
+// dq, dk, dg, dbeta = the sum of the slices' partials, in slice order.
+__global__ void bwd_reduce_kernel(const float* __restrict__ part, float* __restrict__ dq, float* __restrict__ dk,
+                                  float* __restrict__ dg, float* __restrict__ dbeta, size_t rows) {
+    const size_t n4 = rows * (kD / 4);
+    const float4* p4 = reinterpret_cast<const float4*>(part);
+    const size_t stride = rows * (kD / 4);  // one (slice, which) plane in float4
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
+        float4 a[3];
+#pragma unroll
+        for (int w = 0; w < 3; ++w) a[w] = p4[size_t(w) * stride + i];
+#pragma unroll 1
+        for (int s = 1; s < kSlices; ++s) {
+#pragma unroll
+            for (int w = 0; w < 3; ++w) {
+                const float4 x = p4[(size_t(s) * 3 + w) * stride + i];
+                a[w].x += x.x; a[w].y += x.y; a[w].z += x.z; a[w].w += x.w;
+            }
+        }
+        reinterpret_cast<float4*>(dq)[i] = a[0];
+        reinterpret_cast<float4*>(dk)[i] = a[1];
+        reinterpret_cast<float4*>(dg)[i] = a[2];
+    }
+    const float* pb = part + size_t(kSlices) * 3 * rows * kD;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < rows; i += size_t(gridDim.x) * blockDim.x) {
+        float acc = pb[i];
+#pragma unroll 1
+        for (int s = 1; s < kSlices; ++s) acc += pb[size_t(s) * rows + i];
+        dbeta[i] = acc;
+    }
+}
+
+}  // namespace bwd
+
+// checkpoints [B*H][slices][ceil(T/kSub)][cols][rows] fp32, then the slices' partial sums
+// [slices][3][B*T*H][128] and [slices][B*T*H] fp32
+static size_t bwd_ckpt_bytes(int B, int T, int H) {
+    const size_t nsub = (size_t(T) + bwd::kSub - 1) / bwd::kSub;
+    return (size_t(B) * H * bwd::kSlices * nsub * bwd::kSliceCols * kD * sizeof(float) + 255) & ~size_t(255);
+}
+
 size_t recurrent_bwd_workspace_bytes(int B, int T, int H) {
-    const size_t nchunks = (size_t(T) + kC - 1) / kC;
-    return (size_t(B) * H * (nchunks + kC)) * kD * kD * sizeof(float);
+    const size_t rows = size_t(B) * T * H;
+    return bwd_ckpt_bytes(B, T, H) + size_t(bwd::kSlices) * (3 * kD + 1) * rows * sizeof(float);
 }
 
 int launch_recurrent_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          const float* init, const void* dout, const float* dfinal, float* dq, float* dk, float* dv,
                          float* dg, float* dbeta, float* dinit, int B, int Tn, int H, int dtype, float scale,
                          void* ws, size_t ws_bytes, cudaStream_t stream, const char** why) {
+    using namespace bwd;
     const int nbh = B * H;
     if (nbh == 0) return KDA_OK;
     if (ws_bytes < recurrent_bwd_workspace_bytes(B, Tn, H) || ws == nullptr) {
         *why = "workspace smaller than kda_recurrent_bwd_workspace()";
         return KDA_ERR_WORKSPACE;
     }
-    const size_t nchunks = (size_t(Tn) + kC - 1) / kC;
-    float4* ckpt = static_cast<float4*>(ws);
-    float4* scr = ckpt + size_t(nbh) * nchunks * (kD * kD / 4);
+    float* ckpt = static_cast<float*>(ws);
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + bwd_ckpt_bytes(B, Tn, H));
+    const dim3 grid(unsigned(nbh), unsigned(bwd::kSlices));
     if (dtype == KDA_BF16) {
         using Tb = __nv_bfloat16;
-        recurrent_bwd_kernel<Tb><<<nbh, 256, 0, stream>>>(
+        if (!set_smem_attr(recurrent_bwd_kernel<Tb>, smem_bytes<Tb>())) {
+            *why = "cudaFuncSetAttribute failed for the backward kernel";
+            return KDA_ERR_CUDA;
+        }
+        recurrent_bwd_kernel<Tb><<<grid, bwd::kThreads, smem_bytes<Tb>(), stream>>>(
             static_cast<const Tb*>(q), static_cast<const Tb*>(k), static_cast<const Tb*>(v), g, beta, init,
-            static_cast<const Tb*>(dout), dfinal, dq, dk, dv, dg, dbeta, dinit, ckpt, scr, Tn, H, scale);
+            static_cast<const Tb*>(dout), dfinal, dv, dinit, part, ckpt, Tn, H, scale);
     } else {
-        recurrent_bwd_kernel<float><<<nbh, 256, 0, stream>>>(
+        if (!set_smem_attr(recurrent_bwd_kernel<float>, smem_bytes<float>())) {
+            *why = "cudaFuncSetAttribute failed for the backward kernel";
+            return KDA_ERR_CUDA;
+        }
+        recurrent_bwd_kernel<float><<<grid, bwd::kThreads, smem_bytes<float>(), stream>>>(
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), g, beta, init,
-            static_cast<const float*>(dout), dfinal, dq, dk, dv, dg, dbeta, dinit, ckpt, scr, Tn, H, scale);
+            static_cast<const float*>(dout), dfinal, dv, dinit, part, ckpt, Tn, H, scale);
     }
+    const size_t rows = size_t(B) * Tn * H;
+    const unsigned rgrid = unsigned(std::min<size_t>((rows * (kD / 4) + 255) / 256, size_t(148) * 16));
+    bwd_reduce_kernel<<<rgrid, 256, 0, stream>>>(part, dq, dk, dg, dbeta, rows);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         *why = cudaGetErrorString(e);

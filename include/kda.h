@@ -305,19 +305,23 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
  * needs them ("Kimi Linear: An Expressive, Efficient Attention Architecture",
  * section "Training and Inference"; the pages' public-code audit lists
  * q/k/v/g/beta and initial-state gradient tests).  The reverse of each
- * recurrent step is evaluated exactly in fp32 on CUDA cores: one CTA per
- * (sequence, head) runs the forward once storing the state every 64 tokens,
- * then walks the chunks backwards, recomputing each chunk's states.  It is the
- * reference-speed backward (about 2x the token-serial forward work per token);
- * a chunked tensor-core backward is not part of this library.
+ * recurrent step is evaluated exactly in fp32 on CUDA cores.  The recurrence
+ * never mixes value columns, so each (sequence, head) runs as 16 CTAs of 8 value
+ * columns (one key row per thread): each runs the forward storing its state
+ * slice every 16 tokens, then walks the 16-token sub-chunks backwards,
+ * recomputing their states in shared memory.  The slices' partial sums of dq,
+ * dk, dg and dbeta are added by a second kernel in a fixed order, so results are
+ * deterministic.  A chunked tensor-core backward is not part of this library.
  *
  *   q, k, v, d_o   [B,T,H,128], dtype bf16 or fp32 (q, k not normalised here).
  *   g              fp32 [B,T,H,128];  beta fp32 [B,T,H].
  *   initial_state  fp32 [B,H,128,128] or NULL (zero);  d_final_state likewise.
  *   dq, dk, dv, dg fp32 [B,T,H,128];  dbeta fp32 [B,T,H];
  *   d_initial_state fp32 [B,H,128,128] or NULL (not written).
- *   workspace      at least kda_recurrent_bwd_workspace(B, T, H) bytes
- *                  ((ceil(T/64) + 64) x 64 KiB per (sequence, head)), 256-byte aligned.
+ *   workspace      at least kda_recurrent_bwd_workspace(B, T, H) bytes, 256-byte
+ *                  aligned: per (sequence, head), 64 KiB of state checkpoints per
+ *                  16 tokens plus 16 x (3 x 128 + 1) x 4 bytes of partial sums per
+ *                  token (about 28 KiB per token in all).
  * Dense batches only (no cu_seqlens).
  */
 size_t kda_recurrent_bwd_workspace(int B, int T, int H);
