@@ -15,11 +15,10 @@
 //
 // Parallel layout.  The recurrence never mixes value columns: column j of S and
 // of G evolves on its own (y, u, du and dy are per-column).  So every (sequence,
-// head) is split into kSlices = 16 CTAs of kSliceCols = 8 value columns each
-// (small enough that two CTAs share an SM), and a CTA
-// runs the whole sequence for its columns with one key row per thread (128
-// threads): the per-column sums y = S~^T k and du = G^T k are a warp
-// reduce-scatter plus one barrier per token, and the per-row sums dq, dk, dg (and
+// head) is split into kSlices = 16 CTAs of kSliceCols = 8 value columns each, and a
+// CTA is one warp that runs the whole sequence for its columns, lane l holding key
+// rows 4l..4l+3.  The per-column sums y = S~^T k and du = G^T k are a shuffle
+// reduce-scatter inside the warp (no barrier), and the per-row sums dq, dk, dg (and
 // the scalar dbeta) are in-thread partial sums over the CTA's columns.  Those
 // partials go to the workspace and a second kernel adds the slices up (in a fixed
 // order, so results are deterministic); dv and the initial-state gradient are
@@ -38,11 +37,12 @@ namespace bwd {
 constexpr int kSliceCols = 8;                  // value columns per CTA
 constexpr int kSlices = kD / kSliceCols;       // CTAs per (sequence, head)
 constexpr int kSub = 16;                       // tokens per recomputed / staged sub-chunk
-constexpr int kThreads = kD;                   // one key row per thread
+constexpr int kThreads = 32;                   // one warp: lane l holds key rows 4l..4l+3
+constexpr int kRows = kD / kThreads;           // key rows per lane
 constexpr uint32_t kStateBytes = kSub * kSliceCols * kD * sizeof(float);  // states [kSub][col][row]
 
 // One sub-chunk of token inputs in shared memory (element type E of q, k, v, dO):
-// k, q [kSub][128]; g fp32 [kSub][128]; the slice's v, dO [kSub][16]; beta [kSub].
+// k, q [kSub][128]; g fp32 [kSub][128]; the slice's v, dO [kSub][8]; beta [kSub].
 template <typename E>
 struct Stage {
     static constexpr uint32_t K = 0, Q = kSub * kD * sizeof(E), G = 2 * Q, V = G + kSub * kD * 4,
@@ -62,14 +62,13 @@ __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_grou
 __device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Sum x[c] (c < N) over the 32 lanes of the warp.  Returns, in every lane, the full
-// sum of column lane / (32 / N) (groups of 32 / N lanes hold the same column): a
-// reduce-scatter that halves the values per lane at each step, then plain sums.
-template <int N>
-__device__ __forceinline__ float colsum_x32(float (&x)[N], int lane) {
+// Sum x[c] (c < 8) over the 32 lanes of the warp.  Returns, in every lane, the full
+// sum of column lane >> 2 (lanes 4c..4c+3 hold column c): a reduce-scatter that halves
+// the values per lane at each step (7 shuffles), then two plain sums.
+__device__ __forceinline__ float colsum8(float (&x)[8], int lane) {
     int off = 16;
 #pragma unroll
-    for (int half = N / 2; half >= 1; half >>= 1, off >>= 1) {
+    for (int half = 4; half >= 1; half >>= 1, off >>= 1) {
         const bool hi = (lane & off) != 0;
 #pragma unroll
         for (int j = 0; j < half; ++j) {
@@ -79,9 +78,29 @@ __device__ __forceinline__ float colsum_x32(float (&x)[N], int lane) {
         }
     }
     float sum = x[0];
-#pragma unroll
-    for (; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
     return sum;
+}
+
+template <typename T>
+__device__ __forceinline__ void load4(const uint8_t* p, float* out) {  // 4 consecutive elements of type T
+    if constexpr (sizeof(T) == 2) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(p);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        out[0] = __low2float(h2[0]);
+        out[1] = __high2float(h2[0]);
+        out[2] = __low2float(h2[1]);
+        out[3] = __high2float(h2[1]);
+    } else {
+        const float4 f = *reinterpret_cast<const float4*>(p);
+        out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
+    }
+}
+template <typename T>
+__device__ __forceinline__ void load8(const uint8_t* p, float* out) {  // 8 consecutive elements of type T
+    load4<T>(p, out);
+    load4<T>(p + 4 * sizeof(T), out + 4);
 }
 
 template <typename T>
@@ -93,11 +112,10 @@ __global__ void __launch_bounds__(kThreads)
                          float scale) {
     extern __shared__ __align__(128) uint8_t smem[];
     float* sst = reinterpret_cast<float*>(smem);  // [kSub][kSliceCols][kD]: S_{t-1} of the sub-chunk's tokens
-    __shared__ __align__(16) float red[2][4][2][kSliceCols];  // per parity, warp: y and du partials
     using S = Stage<T>;
 
     const int bh = blockIdx.x, sl = blockIdx.y, b = bh / H, h = bh - b * H;
-    const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+    const int lane = threadIdx.x, r0 = kRows * lane;
     const int c0 = sl * kSliceCols;
     const int nsub = (Tn + kSub - 1) / kSub;
     const size_t TH = size_t(gridDim.x) * Tn;  // (sequence, token, head) rows: [B][Tn][H]
@@ -110,13 +128,12 @@ __global__ void __launch_bounds__(kThreads)
     float* ck = ckpt + (size_t(bh) * kSlices + sl) * size_t(nsub) * (kSliceCols * kD);  // [nsub][col][row]
     const uint32_t stage0 = smem_u32(smem + kStateBytes);
 
-    // Stage sub-chunk sc into buffer buf with cp.async (every thread issues its share;
-    // tokens past the end read as zero).  One commit group per call.
+    // Stage sub-chunk sc into buffer buf with cp.async (tokens past the end read as zero).
     auto stage = [&](int sc, int buf, bool with_bwd) {
         const uint32_t base = stage0 + uint32_t(buf) * S::kBytes;
         constexpr int per_row = kD * sizeof(T) / 16;           // 16-byte pieces of a 128-wide row
-        constexpr int per_slice = kSliceCols * sizeof(T) / 16;  // of the slice's 16 values
-        for (int i = r; i < kSub * per_row; i += kThreads) {
+        constexpr int per_slice = kSliceCols * sizeof(T) / 16;  // of the slice's 8 values
+        for (int i = lane; i < kSub * per_row; i += kThreads) {
             const int j = i / per_row, piece = i % per_row, t = sc * kSub + j;
             const bool ok = t < Tn;
             const size_t e = (ok ? row(t) : 0) * kD;
@@ -125,15 +142,15 @@ __global__ void __launch_bounds__(kThreads)
             if (with_bwd)
                 cp_async16(base + S::Q + off, reinterpret_cast<const uint8_t*>(q + e) + piece * 16, ok ? 16u : 0u);
         }
-        for (int i = r; i < kSub * (kD * 4 / 16); i += kThreads) {
+        for (int i = lane; i < kSub * (kD * 4 / 16); i += kThreads) {
             const int j = i / (kD * 4 / 16), piece = i % (kD * 4 / 16), t = sc * kSub + j;
             const bool ok = t < Tn;
             const size_t e = (ok ? row(t) : 0) * kD;
             cp_async16(base + S::G + uint32_t(j * kD * 4 + piece * 16),
                        reinterpret_cast<const uint8_t*>(g + e) + piece * 16, ok ? 16u : 0u);
         }
-        if (r < kSub * per_slice) {
-            const int j = r / per_slice, piece = r % per_slice, t = sc * kSub + j;
+        for (int i = lane; i < kSub * per_slice; i += kThreads) {
+            const int j = i / per_slice, piece = i % per_slice, t = sc * kSub + j;
             const bool ok = t < Tn;
             const size_t e = (ok ? row(t) : 0) * kD + c0;
             const uint32_t off = uint32_t(j * kSliceCols * sizeof(T) + piece * 16);
@@ -142,59 +159,60 @@ __global__ void __launch_bounds__(kThreads)
                 cp_async16(base + S::DO + off, reinterpret_cast<const uint8_t*>(dout + e) + piece * 16,
                            ok ? 16u : 0u);
         }
-        if (r < kSub) {
-            const int t = sc * kSub + r;
+        if (lane < kSub) {
+            const int t = sc * kSub + lane;
             const bool ok = t < Tn;
-            cp_async_4(base + S::B + r * 4, beta + (ok ? row(t) : 0), ok ? 4u : 0u);
+            cp_async_4(base + S::B + lane * 4, beta + (ok ? row(t) : 0), ok ? 4u : 0u);
         }
         cp_commit();
     };
     auto sbuf = [&](int buf) { return smem + kStateBytes + buf * S::kBytes; };
-    auto ld = [&](const uint8_t* p) { return to_f32(*reinterpret_cast<const T*>(p)); };
 
-    auto reduce_cols = [&](float (&x)[kSliceCols], int par, int which) {
-        constexpr int kGroup = 32 / kSliceCols;  // lanes holding one column's sum
-        const float s = colsum_x32<kSliceCols>(x, lane);
-        if (lane % kGroup == 0) red[par][warp][which][lane / kGroup] = s;
-    };
-    auto read_cols = [&](float (&out)[kSliceCols], int par, int which) {
-#pragma unroll
-        for (int c4 = 0; c4 < kSliceCols; c4 += 4) {
-            float4 acc = *reinterpret_cast<const float4*>(&red[par][0][which][c4]);
-#pragma unroll
-            for (int w = 1; w < 4; ++w) {
-                const float4 t4 = *reinterpret_cast<const float4*>(&red[par][w][which][c4]);
-                acc.x += t4.x; acc.y += t4.y; acc.z += t4.z; acc.w += t4.w;
-            }
-            out[c4] = acc.x; out[c4 + 1] = acc.y; out[c4 + 2] = acc.z; out[c4 + 3] = acc.w;
-        }
-    };
-    // one forward step of this thread's row of the slice, token j of staged buffer sb (one barrier)
-    auto fwd_step = [&](float (&s)[kSliceCols], const uint8_t* sb, int j, int par) {
-        const float kr = ld(sb + S::K + (j * kD + r) * sizeof(T));
-        const float a = expf(reinterpret_cast<const float*>(sb + S::G)[j * kD + r]);
-        float yp[kSliceCols];
+    // y[c] (c < 8) = sum over all 128 rows of x[r][c] * w[r]: the warp's column sums, in every lane
+    auto colsums = [&](const float (&x)[kRows][kSliceCols], const float (&w)[kRows], float (&y)[kSliceCols]) {
+        float p[kSliceCols];
 #pragma unroll
         for (int c = 0; c < kSliceCols; ++c) {
-            s[c] *= a;
-            yp[c] = s[c] * kr;
+            p[c] = x[0][c] * w[0];
+#pragma unroll
+            for (int rr = 1; rr < kRows; ++rr) p[c] = fmaf(x[rr][c], w[rr], p[c]);
         }
-        reduce_cols(yp, par, 0);
-        __syncthreads();
-        float y[kSliceCols];
-        read_cols(y, par, 0);
+        const float tot = colsum8(p, lane);
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c) y[c] = __shfl_sync(0xffffffffu, tot, 4 * c);
+    };
+    // the token's per-row k and a = e^g (this lane's 4 rows), from staged buffer sb
+    auto rows_ka = [&](const uint8_t* sb, int j, float (&kr)[kRows], float (&a)[kRows]) {
+        load4<T>(sb + S::K + (j * kD + r0) * sizeof(T), kr);
+        const float4 g4 = *reinterpret_cast<const float4*>(sb + S::G + (j * kD + r0) * 4);
+        a[0] = expf(g4.x); a[1] = expf(g4.y); a[2] = expf(g4.z); a[3] = expf(g4.w);
+    };
+    // one forward step of this lane's 4 rows of the slice, token j of staged buffer sb
+    auto fwd_step = [&](float (&s)[kRows][kSliceCols], const uint8_t* sb, int j) {
+        float kr[kRows], a[kRows], vv[kSliceCols], y[kSliceCols];
+        rows_ka(sb, j, kr, a);
+        load8<T>(sb + S::V + j * kSliceCols * sizeof(T), vv);
         const float bt = reinterpret_cast<const float*>(sb + S::B)[j];
 #pragma unroll
-        for (int c = 0; c < kSliceCols; ++c)
-            s[c] = fmaf(kr, bt * (ld(sb + S::V + (j * kSliceCols + c) * sizeof(T)) - y[c]), s[c]);
+        for (int rr = 0; rr < kRows; ++rr)
+#pragma unroll
+            for (int c = 0; c < kSliceCols; ++c) s[rr][c] *= a[rr];
+        colsums(s, kr, y);
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c) {
+            const float u = bt * (vv[c] - y[c]);
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) s[rr][c] = fmaf(kr[rr], u, s[rr][c]);
+        }
     };
 
     // ---- phase 1: forward, checkpoint at every sub-chunk start
-    float s[kSliceCols];
+    float s[kRows][kSliceCols];
 #pragma unroll
-    for (int c = 0; c < kSliceCols; ++c)
-        s[c] = init ? init[(size_t(bh) * kD + r) * kD + c0 + c] : 0.f;
-    int par = 0;  // parity of the reduction buffer of the next barrier step
+    for (int rr = 0; rr < kRows; ++rr)
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c)
+            s[rr][c] = init ? init[(size_t(bh) * kD + r0 + rr) * kD + c0 + c] : 0.f;
     stage(0, 0, false);
 #pragma unroll 1
     for (int sc = 0; sc < nsub; ++sc) {
@@ -204,25 +222,25 @@ __global__ void __launch_bounds__(kThreads)
         } else {
             cp_wait_0();
         }
-        __syncthreads();  // sub-chunk sc has landed for every thread
+        __syncwarp();  // sub-chunk sc has landed for every lane
         float* dst = ck + size_t(sc) * (kSliceCols * kD);
 #pragma unroll
-        for (int c = 0; c < kSliceCols; ++c) dst[c * kD + r] = s[c];
+        for (int c = 0; c < kSliceCols; ++c)
+            *reinterpret_cast<float4*>(dst + c * kD + r0) = make_float4(s[0][c], s[1][c], s[2][c], s[3][c]);
         const uint8_t* sb = sbuf(sc & 1);
         const int len = min(kSub, Tn - sc * kSub);
 #pragma unroll 1
-        for (int j = 0; j < len; ++j) {
-            fwd_step(s, sb, j, par);
-            par ^= 1;
-        }
-        __syncthreads();  // every thread is done with buffer sc & 1 before it is restaged
+        for (int j = 0; j < len; ++j) fwd_step(s, sb, j);
+        __syncwarp();  // every lane is done with buffer sc & 1 before it is restaged
     }
 
     // ---- phase 2: sub-chunks in reverse; G is the running gradient of the state
-    float G[kSliceCols];
+    float G[kRows][kSliceCols];
 #pragma unroll
-    for (int c = 0; c < kSliceCols; ++c)
-        G[c] = dfinal ? dfinal[(size_t(bh) * kD + r) * kD + c0 + c] : 0.f;
+    for (int rr = 0; rr < kRows; ++rr)
+#pragma unroll
+        for (int c = 0; c < kSliceCols; ++c)
+            G[rr][c] = dfinal ? dfinal[(size_t(bh) * kD + r0 + rr) * kD + c0 + c] : 0.f;
     stage(nsub - 1, (nsub - 1) & 1, true);
 #pragma unroll 1
     for (int sc = nsub - 1; sc >= 0; --sc) {
@@ -232,74 +250,92 @@ __global__ void __launch_bounds__(kThreads)
         } else {
             cp_wait_0();
         }
-        __syncthreads();  // sub-chunk sc has landed for every thread
+        __syncwarp();  // sub-chunk sc has landed for every lane
         const uint8_t* sb = sbuf(sc & 1);
         const int t0 = sc * kSub, len = min(kSub, Tn - t0);
-        {  // recompute S_{t-1} of every token of the sub-chunk into shared memory (own row only)
+        {  // recompute S_{t-1} of every token of the sub-chunk into shared memory (own rows only)
             const float* src = ck + size_t(sc) * (kSliceCols * kD);
 #pragma unroll
-            for (int c = 0; c < kSliceCols; ++c) s[c] = src[c * kD + r];
+            for (int c = 0; c < kSliceCols; ++c) {
+                const float4 x4 = *reinterpret_cast<const float4*>(src + c * kD + r0);
+                s[0][c] = x4.x; s[1][c] = x4.y; s[2][c] = x4.z; s[3][c] = x4.w;
+            }
 #pragma unroll 1
             for (int j = 0; j < len; ++j) {
                 float* dst = sst + j * (kSliceCols * kD);
 #pragma unroll
-                for (int c = 0; c < kSliceCols; ++c) dst[c * kD + r] = s[c];
-                fwd_step(s, sb, j, par);
-                par ^= 1;
+                for (int c = 0; c < kSliceCols; ++c)
+                    *reinterpret_cast<float4*>(dst + c * kD + r0) = make_float4(s[0][c], s[1][c], s[2][c], s[3][c]);
+                fwd_step(s, sb, j);
             }
         }
 #pragma unroll 1
         for (int j = len - 1; j >= 0; --j) {
             const int t = t0 + j;
-            const float kr = ld(sb + S::K + (j * kD + r) * sizeof(T));
-            const float qr = ld(sb + S::Q + (j * kD + r) * sizeof(T)) * scale;
-            const float a = expf(reinterpret_cast<const float*>(sb + S::G)[j * kD + r]);
+            float kr[kRows], a[kRows], qr[kRows], d[kSliceCols], vv[kSliceCols];
+            rows_ka(sb, j, kr, a);
+            load4<T>(sb + S::Q + (j * kD + r0) * sizeof(T), qr);
+            load8<T>(sb + S::DO + j * kSliceCols * sizeof(T), d);
+            load8<T>(sb + S::V + j * kSliceCols * sizeof(T), vv);
             const float bt = reinterpret_cast<const float*>(sb + S::B)[j];
-            float d[kSliceCols];
-#pragma unroll
-            for (int c = 0; c < kSliceCols; ++c) d[c] = ld(sb + S::DO + (j * kSliceCols + c) * sizeof(T));
             const float* src = sst + j * (kSliceCols * kD);
-            float St[kSliceCols], yp[kSliceCols], dup[kSliceCols];
+            float St[kRows][kSliceCols];
 #pragma unroll
             for (int c = 0; c < kSliceCols; ++c) {
-                St[c] = src[c * kD + r] * a;  // S~ = Diag(a) S_{t-1}
-                G[c] = fmaf(qr, d[c], G[c]);
-                yp[c] = St[c] * kr;
-                dup[c] = G[c] * kr;
+                const float4 x4 = *reinterpret_cast<const float4*>(src + c * kD + r0);
+                St[0][c] = x4.x * a[0]; St[1][c] = x4.y * a[1]; St[2][c] = x4.z * a[2]; St[3][c] = x4.w * a[3];
             }
-            reduce_cols(yp, par, 0);
-            reduce_cols(dup, par, 1);
-            __syncthreads();
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+                const float qs = qr[rr] * scale;
+#pragma unroll
+                for (int c = 0; c < kSliceCols; ++c) G[rr][c] = fmaf(qs, d[c], G[rr][c]);
+            }
             float y[kSliceCols], du[kSliceCols];
-            read_cols(y, par, 0);
-            read_cols(du, par, 1);
-            par ^= 1;
-            float udo = 0.f, dbt = 0.f, xq = 0.f, xk = 0.f, xg = 0.f, dur = 0.f;
+            colsums(St, kr, y);
+            colsums(G, kr, du);
+            float udo = 0.f, dbt = 0.f, u[kSliceCols], dy[kSliceCols];
 #pragma unroll
             for (int c = 0; c < kSliceCols; ++c) {
-                const float rr = ld(sb + S::V + (j * kSliceCols + c) * sizeof(T)) - y[c];  // v - y
-                const float u = bt * rr, dy = -bt * du[c];
-                udo = fmaf(u, d[c], udo);
+                const float rr = vv[c] - y[c];  // v - y
+                u[c] = bt * rr;
+                dy[c] = -bt * du[c];
+                udo = fmaf(u[c], d[c], udo);
                 dbt = fmaf(du[c], rr, dbt);
-                xq = fmaf(St[c], d[c], xq);
-                xk = fmaf(G[c], u, fmaf(St[c], dy, xk));
-                const float gt = fmaf(kr, dy, G[c]);  // G~ = G + k dy^T
-                xg = fmaf(gt, St[c], xg);
-                G[c] = gt * a;  // G <- Diag(a) G~
-                dur = (c == r) ? du[c] : dur;
+            }
+            float xq[kRows], xk[kRows], xg[kRows];
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+                float aq = 0.f, ak = 0.f, ag = 0.f;
+#pragma unroll
+                for (int c = 0; c < kSliceCols; ++c) {
+                    aq = fmaf(St[rr][c], d[c], aq);
+                    ak = fmaf(G[rr][c], u[c], fmaf(St[rr][c], dy[c], ak));
+                    const float gt = fmaf(kr[rr], dy[c], G[rr][c]);  // G~ = G + k dy^T
+                    ag = fmaf(gt, St[rr][c], ag);
+                    G[rr][c] = gt * a[rr];  // G <- Diag(a) G~
+                }
+                xq[rr] = scale * (aq + kr[rr] * udo);
+                xk[rr] = ak;
+                xg[rr] = ag;
             }
             const size_t e = row(t);
-            if (r < kSliceCols) dv[e * kD + c0 + r] = bt * dur;  // dv = beta du: thread r < kSliceCols writes column c0 + r
-            if (r == 0) p_db[e] = dbt;
-            p_dq[e * kD + r] = scale * (xq + kr * udo);
-            p_dk[e * kD + r] = xk;
-            p_dg[e * kD + r] = xg;
+            float dur = 0.f;
+#pragma unroll
+            for (int c = 0; c < kSliceCols; ++c) dur = (c == lane) ? du[c] : dur;
+            if (lane < kSliceCols) dv[e * kD + c0 + lane] = bt * dur;  // dv = beta du: lane c writes column c0 + c
+            if (lane == 0) p_db[e] = dbt;
+            *reinterpret_cast<float4*>(p_dq + e * kD + r0) = make_float4(xq[0], xq[1], xq[2], xq[3]);
+            *reinterpret_cast<float4*>(p_dk + e * kD + r0) = make_float4(xk[0], xk[1], xk[2], xk[3]);
+            *reinterpret_cast<float4*>(p_dg + e * kD + r0) = make_float4(xg[0], xg[1], xg[2], xg[3]);
         }
-        __syncthreads();  // every thread is done with buffer sc & 1 before it is restaged
+        __syncwarp();  // every lane is done with buffer sc & 1 before it is restaged
     }
     if (dinit) {
 #pragma unroll
-        for (int c = 0; c < kSliceCols; ++c) dinit[(size_t(bh) * kD + r) * kD + c0 + c] = G[c];
+        for (int rr = 0; rr < kRows; ++rr)
+#pragma unroll
+            for (int c = 0; c < kSliceCols; ++c) dinit[(size_t(bh) * kD + r0 + rr) * kD + c0 + c] = G[rr][c];
     }
 }
 

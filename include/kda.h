@@ -306,8 +306,8 @@ int kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *
  * section "Training and Inference"; the pages' public-code audit lists
  * q/k/v/g/beta and initial-state gradient tests).  The reverse of each
  * recurrent step is evaluated exactly in fp32 on CUDA cores.  The recurrence
- * never mixes value columns, so each (sequence, head) runs as 16 CTAs of 8 value
- * columns (one key row per thread): each runs the forward storing its state
+ * never mixes value columns, so each (sequence, head) runs as 16 one-warp CTAs of
+ * 8 value columns (lane l holds key rows 4l..4l+3): each runs the forward storing its state
  * slice every 16 tokens, then walks the 16-token sub-chunks backwards,
  * recomputing their states in shared memory.  The slices' partial sums of dq,
  * dk, dg and dbeta are added by a second kernel in a fixed order, so results are
