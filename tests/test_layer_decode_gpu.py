@@ -3,7 +3,8 @@ outputs, and kda_layer_decode continuing the sequences from them.
 
 Each sequence is run by the fp64 oracle layer in one pass over all its tokens
 (prompt, then the decoded tokens); the GPU runs a prefill and then decode calls
-from the cache.  Tolerances as in test_layer_gpu.py (y 2e-2, state 1e-2)."""
+from the cache.  Tolerances as in test_layer_gpu.py: relative L2 1e-2 on y and on
+the state."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +14,7 @@ import synth
 from helpers import f64, rel_l2
 
 pytestmark = pytest.mark.gpu
-TOL_Y = 2e-2
+TOL_Y = 1e-2
 TOL_S = 1e-2
 
 

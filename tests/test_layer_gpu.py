@@ -1,14 +1,15 @@
 """kda_layer_fwd vs the fp64 oracle layer.
 
-The GPU path rounds every intermediate activation to bf16 (the projection
-outputs, q/k/v after the convolution, the gate and norm inputs, the KDA
-output), each a relative error of about 2^-9, while the oracle keeps fp64
-throughout.  Two effects then add up on y: the operator's own 1e-2 budget,
-and the per-(token, head) RMSNorm, which rescales every row of the KDA
-output to unit RMS -- so rows whose value is a small result of cancellation
-(early tokens of a sequence, where o ~ beta (k.q) v with k.q ~ 1/sqrt(128))
-carry their larger relative error into y at full weight.  Tolerance: relative
-L2 <= 2e-2 on y, 1e-2 on the final state (the operator's bar)."""
+The GPU path rounds the layer's activations to bf16 (the projection outputs,
+q/k/v after the convolution, the normed output), each a relative error of
+about 2^-9, while the oracle keeps fp64 throughout; the operator's output, the
+decay input and the gate input stay fp32 into the GEMM epilogues that use them.
+The per-(token, head) RMSNorm carries each row's relative error into y at full
+weight, and for rows whose RMS is far below the norm's epsilon (the first
+tokens of a sequence, o ~ beta (k.q) v) absolute errors pass straight through,
+so the shortest sequences sit closest to the bar (about 9e-3 for 4 tokens).
+Tolerance: relative L2 <= 1e-2 on y and on the final state (the benchmark spec's
+bar for outputs and states)."""
 import numpy as np
 import pytest
 import torch
