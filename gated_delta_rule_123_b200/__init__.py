@@ -29,7 +29,7 @@ SYMBOLS = (
     "kda_gdn_chunk_fwd", "kda_recurrent_fwd", "kda_layer_decode_workspace", "kda_layer_decode",
     "kda_dplr_chunk_fwd_workspace", "kda_dplr_chunk_fwd", "kda_recurrent_bwd_workspace", "kda_recurrent_bwd",
     "kda_chunk_fwd_segment_tokens", "kda_chunk_fwd_workspace_min", "kda_debug_fault_injection",
-    "kda_linear_bf16",
+    "kda_linear_bf16", "kda_chunk_fwd_plan_items",
 )
 
 
@@ -62,6 +62,8 @@ def _load():
     lib.kda_chunk_fwd_workspace_min.restype = sz
     lib.kda_chunk_fwd_segment_tokens.argtypes = [i, i, i, i, ctypes.POINTER(ctypes.c_int)]
     lib.kda_chunk_fwd_segment_tokens.restype = i
+    lib.kda_chunk_fwd_plan_items.argtypes = [vp, i, i, i, i, ctypes.POINTER(ctypes.c_int), i]
+    lib.kda_chunk_fwd_plan_items.restype = i
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i
     lib.kda_gdn_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
@@ -156,10 +158,22 @@ _trace_keep = None
 
 
 def chunk_fwd_segments(B, T, H, num_seqs=0):
-    """(first segment tokens, following segment tokens) of a kda_chunk_fwd call; (0, 0) if unsegmented."""
+    """(first segment tokens, following segment tokens) of a kda_chunk_fwd call; (0, 0) if unsegmented,
+    (-1, -1) if the device plans the cuts from cu_seqlens (see chunk_fwd_plan)."""
     mid = ctypes.c_int(0)
     first = int(_lib.kda_chunk_fwd_segment_tokens(B, T, H, num_seqs, ctypes.byref(mid)))
     return first, mid.value
+
+
+def chunk_fwd_plan(workspace, B, T, H, num_seqs=0):
+    """The segments the last chunk_fwd call with this workspace and these sizes
+    ran: a list of (sequence, first token, end token, g, G).  Waits for the device."""
+    cap = 4096
+    rows = (ctypes.c_int * (5 * cap))()
+    n = int(_lib.kda_chunk_fwd_plan_items(ctypes.c_void_p(workspace.data_ptr()), B, T, H, num_seqs, rows, cap))
+    if n < 0:
+        raise KDAError(KDA_ERR_CUDA, "kda_chunk_fwd_plan_items", "copy failed")
+    return [tuple(rows[5 * i: 5 * i + 5]) for i in range(min(n, cap))]
 
 
 def chunk_fwd_workspace_bytes(B, T, H, num_seqs=0, dtype=KDA_BF16, l2norm_qk=False) -> int:

@@ -18,6 +18,7 @@ int launch_recurrent_bwd(const void* q, const void* k, const void* v, const floa
                          float* dg, float* dbeta, float* dinit, int B, int Tn, int H, int dtype, float scale,
                          void* ws, size_t ws_bytes, cudaStream_t stream, const char** why);
 int chunk_segment_tokens(int B, int T, int H, int num_seqs, int* middle);
+int chunk_plan_items(const void* ws, int B, int T, int H, int num_seqs, int* rows, int max_rows);
 size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm);
 int launch_recurrent_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* state, void* o, int B, int Tn, int H, int dtype, float scale, int l2norm,
@@ -104,6 +105,11 @@ int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int* middle_
     if (middle_tokens) *middle_tokens = 0;
     if (B < 0 || T < 0 || H < 0 || num_seqs < 0) return 0;
     return chunk_segment_tokens(B, T, H, num_seqs, middle_tokens);
+}
+
+int kda_chunk_fwd_plan_items(const void* workspace, int B, int T, int H, int num_seqs, int* rows, int max_rows) {
+    if (!workspace || !rows || max_rows < 0 || B < 0 || T < 0 || H < 0 || num_seqs < 0) return -1;
+    return chunk_plan_items(workspace, B, T, H, num_seqs, rows, max_rows);
 }
 
 size_t kda_chunk_fwd_workspace_min(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk) {

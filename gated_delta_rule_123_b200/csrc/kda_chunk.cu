@@ -56,7 +56,8 @@ struct SegItem {
     int g;          // segment index inside the sequence
     int G;          // number of segments of the sequence
     int first;      // item index of segment 0 of the sequence
-    int pad0, pad1;
+    int slot;       // product-image slot of its chunk 0 (chunk c of the segment uses slot + c)
+    int pad1;
 };
 
 // Optional per-stage cycle counters, compiled in only with -DKDA_STAGE_TIMING for
@@ -126,8 +127,7 @@ static_assert(PI_QP - PI_WN == OFF_QP - OFF_WN && PI_KM - PI_P == OFF_KM - OFF_P
 
 struct ChunkArgs {
     const float* beta;
-    uint8_t* prod;    // product images [item][prodL][H] (segmented calls)
-    int prodL;        // chunk slots per item
+    uint8_t* prod;    // product images [slot][H] (segmented calls; SegItem::slot)
     const float* gs;  // per-head scalar log-gates [Ttot][H] (scalar-gate kernels only)
     const float* init_state;
     float* final_state;
@@ -137,6 +137,9 @@ struct ChunkArgs {
     float* segN;
     float* segX;
     float* segS;  // per-segment start states (phase 1 writes segment 1's, the combine pass the rest)
+    const int* order;    // balanced plans: the launch order of the items (heaviest first), else null
+    const int* n_order;  // the number of items in that order
+    int seg0_whole;      // balanced plans: segment 0 runs its output in phase 1 from the initial state
     int H;
     float scale;
 };
@@ -215,7 +218,7 @@ constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per col
 template <bool kSummary, typename OutT, bool kScalarGate>
 __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                            const CUtensorMap& tm_g, const CUtensorMap& tm_o, const ChunkArgs& p,
-                                           const SegItem it) {
+                                           const SegItem it, const int item_id, const int h) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw;
     const uint32_t sbase = smem_u32(sm);
@@ -227,7 +230,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
     constexpr bool kStageO = sizeof(OutT) == 2;  // bf16 output leaves through TMA stores
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, part = warp >> 2;  // TMEM lane quadrant; column quarter
-    const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
+    const int H = p.H;
 
     float* sBeta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64] beta per chunk parity
     float* sFrOp = sBeta2 + 128;                               // [128] post(prev) * e^{mp}
@@ -580,7 +583,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 #endif
         KDA_STAGE(1);
         // the map pass exports what the output pass of this segment reuses
-        uint8_t* img = (kSummary && p.prod) ? p.prod + ((size_t(item_id) * p.prodL + c) * H + h) * kProdBytes : nullptr;
+        uint8_t* img = (kSummary && p.prod) ? p.prod + ((size_t(it.slot) + c) * H + h) * kProdBytes : nullptr;
         if (img) {
             if (tid == kExporter) {  // Qp and Km of this chunk are final (built before the last barrier)
                 bulk_store_1d(img + PI_QP, sm + OFF_QP, 16384u);
@@ -1103,6 +1106,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
         } else if (it.g == it.G - 1) {
             if (p.final_state) dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
+        } else if (p.seg0_whole && it.g == 0 && item_id + 1 < *p.n_items) {  // the start state of segment 1
+            dstS = p.segS + (size_t(item_id + 1) * H + h) * (kD * kD);
         }
         tc_fence_after();
         auto store = [&](uint32_t tcol, float* dst) {
@@ -1168,7 +1173,7 @@ static_assert(MISC + 256 <= kSmemBytes && (2 * kProdBytes) % 1024 == 0, "light s
 
 template <typename OutT>
 __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const CUtensorMap& tm_o, const ChunkArgs& p,
-                                                 const SegItem it) {
+                                                 const SegItem it, const int item_id, const int h) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw;
     const uint32_t sbase = smem_u32(sm);
@@ -1179,7 +1184,7 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
     constexpr bool kStageO = sizeof(OutT) == 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, part = warp >> 2;
-    const int item_id = blockIdx.x, h = blockIdx.y, H = p.H;
+    const int H = p.H;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + light::MISC);  // [0],[1]: buffer loads; [2]: MMA
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
     constexpr int kLoader = 96;
@@ -1206,7 +1211,7 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
     const int vrow = quad * 32 + lane;
     const int t_begin = it.tok_begin, t_end = it.tok_end;
     const int nchunks = (t_end - t_begin + kC - 1) / kC;
-    auto image = [&](int c) { return p.prod + ((size_t(item_id) * p.prodL + c) * H + h) * kProdBytes; };
+    auto image = [&](int c) { return p.prod + ((size_t(it.slot) + c) * H + h) * kProdBytes; };
     auto issue = [&](int c) {  // chunk c's image and V into buffer c & 1
         const int b = c & 1;
         mbar_arrive_expect_tx(&bars[b], kProdBytes + 16384u);
@@ -1388,21 +1393,43 @@ __device__ __forceinline__ void chunk_light_body(const CUtensorMap& tm_v, const 
     if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
+// The (item, head) pair a CTA of a phase launch runs; false when it has none.
+// Uniform plans map blockIdx.x to the item and blockIdx.y to the head.  Balanced
+// plans list their items heaviest first, and consecutive CTAs (in launch order)
+// take the heads of one item in turn: the longest items start first and the
+// shorter ones fill the SMs that free up.
+__device__ __forceinline__ bool cta_item(const ChunkArgs& p, int& item, int& h) {
+    if (p.order) {
+        const int lin = int(blockIdx.x + blockIdx.y * gridDim.x);
+        const int r = lin / p.H;
+        if (r >= *p.n_order) return false;
+        item = p.order[r];
+        h = lin - r * p.H;
+        return true;
+    }
+    item = int(blockIdx.x);
+    h = int(blockIdx.y);
+    return item < *p.n_items;
+}
+
 // Phase 1 (and the only launch of an unsegmented call): the maps of every
 // segment of a segmented sequence (the last segment's map only exports its chunk
 // products, and runs only when there is room for them), and the whole output of
-// an unsegmented one.  Segmented calls thus run one code path on every SM.
+// an unsegmented one.  Segmented calls of a uniform plan thus run one code path
+// on every SM.  In a balanced plan segment 0 needs no map: it runs its output
+// from the initial state here and leaves its end state as segment 1's start.
 template <typename OutT, bool kScalarGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
-    if (int(blockIdx.x) >= *p.n_items) return;
-    const SegItem it = p.items[blockIdx.x];
-    if (it.G == 1)
-        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+    int item, h;
+    if (!cta_item(p, item, h)) return;
+    const SegItem it = p.items[item];
+    if (it.G == 1 || (p.seg0_whole && it.g == 0))
+        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
     else if (it.g < it.G - 1 || p.prod)
-        chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+        chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
 }
 
 // Phase 2: the outputs of every segment of a segmented sequence from its start
@@ -1413,13 +1440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
-    if (int(blockIdx.x) >= *p.n_items) return;
-    const SegItem it = p.items[blockIdx.x];
-    if (it.G == 1) return;  // its output was written in phase 1
+    int item, h;
+    if (!cta_item(p, item, h)) return;
+    const SegItem it = p.items[item];
+    if (it.G == 1 || (p.seg0_whole && it.g == 0)) return;  // its output was written in phase 1
     if (p.prod)
-        chunk_light_body<OutT>(tm_v, tm_o, p, it);
+        chunk_light_body<OutT>(tm_v, tm_o, p, it, item, h);
     else
-        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it);
+        chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
 }
 
 // ---------------------------------------------------------------- plan
@@ -1460,7 +1488,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
                 s.g = g;
                 s.G = G;
                 s.first = off;
-                s.pad0 = s.pad1 = 0;
+                s.slot = L < (1 << 30) ? id * L : 0;  // image slots exist only in segmented plans
+                s.pad1 = 0;
                 items[id] = s;
             }
         }
@@ -1471,10 +1500,201 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, in
     if (threadIdx.x == 0) *n_items = min(s_base, max_items);
 }
 
+// ---------------------------------------------------------------- balanced plan
+// Packed sequences whose (sequence, head) pairs are too many for the uniform plan
+// (which cuts every sequence into G equal segments, G CTAs per pair) but whose
+// lengths differ: unsegmented, the longest sequence alone sets the time while
+// most SMs idle.  The balanced plan cuts each sequence at a common target
+// length lam: segment 0 runs its output from the initial state in phase 1 (no
+// map, no second pass), the later ones run a map in phase 1 and an output pass
+// in phase 2, and short sequences stay whole.  lam is chosen on the device, from
+// the lengths in cu_seqlens, among 16 candidates (one warp each), by a closed-form
+// estimate of each phase's time: the longer of its longest CTA and its mean load
+// per SM plus half a mean CTA (the tail), plus the combine pass's waves.  The
+// launch order puts the longest items first, so shorter ones fill the SMs that
+// free up.
+constexpr int kBalMaxSeqs = 64;    // sequences a balanced plan takes
+constexpr int kBalMaxItems = 128;  // segments it may cut them into
+constexpr int kBalMinChunks = 16;  // shortest target segment length
+constexpr int kBalCands = 16;      // target lengths tried: ceil(longest / (w + 1)), w < 16
+
+// Costs that the plan weighs, in thousands of SM cycles on B200 (fitted to the
+// phase times of 24 plans over three length mixes, all SMs busy).
+struct BalCost {
+    float whole;  // per chunk of an output pass from a known start state (segment 0, whole sequences)
+    float map;    // per chunk of a map pass
+    float item;   // per phase-1 CTA: TMEM and barriers, the start state in, the end state out
+    float light;  // per chunk of a later segment's output pass
+    float litem;  // per phase-2 CTA
+    float comb;   // per combine step of one CTA (sequence, head, 16 columns), SMs full
+    float seg;    // the extra launches' cost when anything is cut
+};
+
+// Cuts a sequence of n chunks at target length lam: segment 0 takes l0 chunks
+// (r = map / whole cost: as long as a map of the others' length takes), the
+// others lm (the last one the rest).  Returns the segment count G <= ceil(n/lam).
+__device__ __forceinline__ int bal_split(int n, int lam, float r, int& l0, int& lm) {
+    if (n <= lam) {
+        l0 = n;
+        lm = 0;
+        return 1;
+    }
+    const int G0 = (n + lam - 1) / lam;
+    l0 = int(roundf(float(n) * r / (r + float(G0 - 1))));
+    l0 = max(1, min(l0, n - 1));
+    const int rest = n - l0;
+    lm = (rest + G0 - 2) / (G0 - 1);
+    return 1 + (rest + lm - 1) / lm;
+}
+
+// One CTA of 512 threads (16 warps), N <= kBalMaxSeqs.  Warp w scores the target
+// length of candidate w; then the best one (ties to the longer length) is cut and
+// written: the segment table in sequence order (segments of a sequence adjacent,
+// as the combine pass expects), each sequence's first item, the phase-1 launch
+// order (all items, heaviest first), the phase-2 launch order (segments g >= 1,
+// longest first) and the two counts.
+__global__ void __launch_bounds__(32 * kBalCands) plan_balanced_kernel(const int32_t* cu, int N, int H, int nsm,
+                                                                       BalCost cost, int max_items, SegItem* items,
+                                                                       int* counts, int* seq_first, int* order1,
+                                                                       int* order2) {
+    __shared__ int s_n[kBalMaxSeqs], s_off[kBalMaxSeqs + 1];
+    __shared__ unsigned long long s_key[kBalCands];
+    __shared__ float s_k1[kBalMaxItems], s_k2[kBalMaxItems];
+    __shared__ int s_maxn, s_lam, s_total;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp == 0) {
+        int mx = 0;
+        for (int n = lane; n < N; n += 32) {
+            const int c = (cu[n + 1] - cu[n] + kC - 1) / kC;
+            s_n[n] = c;
+            mx = max(mx, c);
+        }
+        mx = int(__reduce_max_sync(0xffffffffu, unsigned(mx)));
+        if (lane == 0) s_maxn = mx;
+    }
+    __syncthreads();
+    const int maxn = s_maxn;
+    const float r = cost.map / cost.whole;
+    const int cap = min(max_items, kBalMaxItems);
+    {  // this warp's candidate: sums and maxima of both phases' CTA costs
+        const int w = warp;
+        const int lam = max(kBalMinChunks, (maxn + w) / (w + 1));
+        const bool repeat = w > 0 && lam == max(kBalMinChunks, (maxn + w - 1) / w);
+        float sum1 = 0.f, max1 = 0.f, sum2 = 0.f, max2 = 0.f;
+        int n1 = 0, n2 = 0, maxG = 1, steps = 0;
+        for (int n = lane; n < N; n += 32) {
+            int l0, lm;
+            const int nch = s_n[n];
+            const int G = bal_split(nch, lam, r, l0, lm);
+            const float c0 = float(G == 1 ? nch : l0) * cost.whole + cost.item;
+            sum1 += c0;
+            max1 = fmaxf(max1, c0);
+            for (int g = 1; g < G; ++g) {
+                const int len = min(lm, nch - l0 - (g - 1) * lm);
+                const float cm = float(len) * cost.map + cost.item, cl = float(len) * cost.light + cost.litem;
+                sum1 += cm;
+                max1 = fmaxf(max1, cm);
+                sum2 += cl;
+                max2 = fmaxf(max2, cl);
+            }
+            n1 += G;
+            n2 += G - 1;
+            maxG = max(maxG, G);
+            steps += max(0, G - 2);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
+            sum2 += __shfl_xor_sync(0xffffffffu, sum2, off);
+            max1 = fmaxf(max1, __shfl_xor_sync(0xffffffffu, max1, off));
+            max2 = fmaxf(max2, __shfl_xor_sync(0xffffffffu, max2, off));
+        }
+        n1 = __reduce_add_sync(0xffffffffu, n1);
+        n2 = __reduce_add_sync(0xffffffffu, n2);
+        maxG = __reduce_max_sync(0xffffffffu, maxG);
+        steps = __reduce_add_sync(0xffffffffu, steps);
+        float est = 3.0e38f;
+        if (!repeat && n1 <= cap) {
+            const float per_sm = float(H) / float(nsm);
+            est = fmaxf(max1, sum1 * per_sm + 0.5f * sum1 / float(n1));
+            if (n2 > 0) {  // the combine runs H x 8 CTAs per chained sequence: waves of nsm
+                const int waves = max(maxG - 2, (steps * H * (kD / 16) + nsm - 1) / nsm);
+                est += fmaxf(max2, sum2 * per_sm + 0.5f * sum2 / float(n2)) + cost.comb * float(waves) + cost.seg;
+            }
+        }
+        // the lowest estimate, ties to the lowest w (the longest target length)
+        if (lane == 0) s_key[w] = (static_cast<unsigned long long>(__float_as_uint(est)) << 32) | unsigned(lam);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        unsigned long long best = s_key[0];
+        for (int w = 1; w < kBalCands; ++w)
+            if ((s_key[w] >> 32) < (best >> 32)) best = s_key[w];
+        s_lam = int(best & 0xffffffffu);
+    }
+    __syncthreads();
+    const int lam = s_lam;
+    int G = 0, l0 = 0, lm = 0, nch = 0;
+    if (tid < N) {
+        nch = s_n[tid];
+        G = bal_split(nch, lam, r, l0, lm);
+        s_off[tid] = G;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int off = 0;
+        for (int n = 0; n < N; ++n) {
+            const int g = s_off[n];
+            s_off[n] = off;
+            off += g;
+        }
+        s_off[N] = off;
+        s_total = min(off, cap);
+    }
+    __syncthreads();
+    const int total = s_total;
+    if (tid < N) {
+        const int off = s_off[tid], sb = cu[tid], se = cu[tid + 1];
+        seq_first[tid] = off;
+        for (int g = 0; g < G && off + g < total; ++g) {
+            const int c0 = g == 0 ? 0 : l0 + (g - 1) * lm;
+            const int c1 = g == 0 ? (G == 1 ? nch : l0) : min(nch, c0 + lm);
+            SegItem s;
+            s.seq = tid;
+            s.tok_begin = min(se, sb + c0 * kC);
+            s.tok_end = min(se, sb + c1 * kC);
+            s.g = g;
+            s.G = G;
+            s.first = off;
+            s.slot = sb / kC + tid + c0;  // distinct for every chunk of every sequence
+            s.pad1 = 0;
+            items[off + g] = s;
+            s_k1[off + g] = float(c1 - c0) * (g == 0 ? cost.whole : cost.map);
+            s_k2[off + g] = g == 0 ? -1.f : float(c1 - c0);
+        }
+    }
+    __syncthreads();
+    if (tid < total) {  // ranks: heavier first, ties in item order
+        const float a = s_k1[tid], b = s_k2[tid];
+        int r1 = 0, r2 = 0;
+        for (int j = 0; j < total; ++j) {
+            r1 += (s_k1[j] > a) || (s_k1[j] == a && j < tid);
+            r2 += s_k2[j] >= 0.f && ((s_k2[j] > b) || (s_k2[j] == b && j < tid));
+        }
+        order1[r1] = tid;
+        if (b >= 0.f) order2[r2] = tid;
+    }
+    if (tid == 0) {
+        counts[0] = total;
+        counts[1] = total - N;
+    }
+}
+
 // ---------------------------------------------------------------- combine
 // Chains the segment maps of one (sequence, head, 16-column slice):
 // S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1 (segment 0
-// gets the initial state).  X_g^T (64 KB, written transposed by the summary
+// gets the initial state).  With s0 = 1 (balanced plans) phase 1 has already
+// written S_1, the end state of segment 0's output pass, and the chain starts there.  X_g^T (64 KB, written transposed by the summary
 // pass) streams into shared memory with 1-D bulk copies, double-buffered.  Two
 // halves of 256 threads each sum over half of the key dimension, a thread owning
 // a 2 x 4 tile of the slice; the halves' sums meet in shared memory.
@@ -1486,13 +1706,13 @@ constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 256 * 8 * 4 + 64
 __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem* items, const int* n_items,
                                                                   const int* seq_first, int N, const float* init,
                                                                   const float* segN, const float* segXt,
-                                                                  float* segS, int H) {
+                                                                  float* segS, int H, int s0) {
     const int n = blockIdx.x, h = blockIdx.y, z = blockIdx.z;  // one CTA per (sequence, head, slice)
     if (n >= N) return;
     const int item = seq_first[n];
     if (item < 0 || item >= *n_items) return;
     const SegItem it = items[item];
-    if (it.g != 0 || it.G < 2) return;
+    if (it.g != 0 || it.G < 2 + s0) return;
     extern __shared__ __align__(128) uint8_t csm[];
     float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
     float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
@@ -1509,22 +1729,27 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem*
         fence_mbar_init();
     }
     __syncthreads();
-    // step j = 0, 1, ..., G-2 maps S_j to S_{j+1} with segment j's map (S_0 = the initial state)
+    // step j = 0, 1, ..., G-2-s0 maps S_{s0+j} to S_{s0+j+1} with segment s0+j's map
+    // (S_0 = the initial state; S_1 = segment 0's end state when s0 = 1)
     auto fetch = [&](int j) {
         mbar_arrive_expect_tx(&bar[j & 1], 65536u);
-        bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + j) * H * (kD * kD) + hs, 65536u, &bar[j & 1]);
+        bulk_load_1d(sX + (j & 1) * kD * kD, segXt + size_t(item + s0 + j) * H * (kD * kD) + hs, 65536u,
+                     &bar[j & 1]);
     };
     if (tid == 0) fetch(0);
+    const float* s_in = s0 ? segS + size_t(item + 1) * H * (kD * kD) + hs
+                           : (init ? init + size_t(it.seq) * H * (kD * kD) + hs : nullptr);
     for (int e = tid; e < kD * kCombCols; e += kCombThreads) {
         const int kk = e / kCombCols, jj = e % kCombCols;
-        sS[e] = init ? init[size_t(it.seq) * H * (kD * kD) + hs + size_t(kk) * kD + c0 + jj] : 0.f;
+        sS[e] = s_in ? s_in[size_t(kk) * kD + c0 + jj] : 0.f;
     }
     __syncthreads();
+    const int steps = it.G - 1 - s0;
     bool ok = true;
     int fetched = 1, j = 0;  // fetches issued (thread 0) and the step being consumed
-    for (; j + 1 < it.G; ++j) {
-        const int g = j;  // the segment whose map this step applies
-        if (tid == 0 && j + 2 < it.G) {
+    for (; j < steps; ++j) {
+        const int g = s0 + j;  // the segment whose map this step applies
+        if (tid == 0 && j + 1 < steps) {
             fetch(j + 1);
             fetched = j + 2;
         }
@@ -1645,12 +1870,18 @@ struct ChunkPlan {
     int N, L, max_items;
     long long Ttot;
     bool scan;
-    size_t off_items, off_count, off_first, off_segN, off_segX, off_segS, off_q, off_k, off_v, total;
+    bool balanced;  // per-sequence cuts chosen on the device (plan_balanced_kernel)
+    size_t off_items, off_count, off_first, off_order1, off_order2, off_segN, off_segX, off_segS, off_q, off_k,
+        off_v, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+constexpr size_t kPlanHead = 16;  // the item counts
 
-ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2norm, bool varlen, int nsm) {
+// balanced_ok = false leaves packed calls with many pairs unsegmented (for workspaces
+// too small for the balanced plan's per-segment states).
+ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2norm, bool varlen, int nsm,
+                          bool balanced_ok = true) {
     ChunkPlan pl{};
     pl.N = varlen ? num_seqs : B;
     pl.Ttot = varlen ? (long long)T : (long long)B * T;
@@ -1670,10 +1901,22 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     pl.L0 = L0;
     pl.scan = L < (1 << 30);
     pl.max_items = int(pl.N + (pl.scan ? (chunks_bound + L - 1) / L : 0));
-    size_t off = 0;
+    // Packed sequences with too many pairs for the uniform plan: the balanced plan,
+    // when the call is long enough for some sequence to be cut.  It makes at most
+    // sum_n ceil(chunks_n / kBalMinChunks) <= N + chunks_bound / kBalMinChunks segments.
+    if (balanced_ok && !pl.scan && varlen && pairs > 0 && pl.N <= kBalMaxSeqs &&
+        (pl.Ttot + kC - 1) / kC > kBalMinChunks) {
+        const long long bound = pl.N + (chunks_bound + kBalMinChunks - 1) / kBalMinChunks;
+        pl.balanced = true;
+        pl.scan = true;
+        pl.max_items = int(bound < kBalMaxItems ? bound : kBalMaxItems);
+    }
+    size_t off = 0;  // the counts and the segment table first, where every plan has them
+    pl.off_count = off; off = up256(off + kPlanHead);
     pl.off_items = off; off = up256(off + sizeof(SegItem) * size_t(pl.max_items));
-    pl.off_count = off; off = up256(off + 16);
     pl.off_first = off; off = up256(off + (pl.scan ? sizeof(int) * size_t(pl.N) : 0));
+    pl.off_order1 = off; off = up256(off + (pl.balanced ? sizeof(int) * size_t(pl.max_items) : 0));
+    pl.off_order2 = off; off = up256(off + (pl.balanced ? sizeof(int) * size_t(pl.max_items) : 0));
     const size_t st = size_t(pl.max_items) * H * kD * kD * sizeof(float);
     pl.off_segN = off; off = up256(off + (pl.scan ? st : 0));
     pl.off_segX = off; off = up256(off + (pl.scan ? st : 0));
@@ -1684,7 +1927,9 @@ ChunkPlan make_chunk_plan(int B, int T, int H, int num_seqs, int dtype, int l2no
     pl.off_k = off; off = up256(off + (need_qk ? tok : 0));
     pl.off_v = off; off = up256(off + (dtype == KDA_FP32 ? tok : 0));
     pl.total_min = off;
-    pl.prod_bytes = pl.scan ? size_t(pl.max_items) * size_t(L) * H * kProdBytes : 0;
+    // image slots: L per item in a uniform plan; one per chunk of the call in a balanced one
+    const size_t slots = pl.balanced ? size_t(chunks_bound) : size_t(pl.max_items) * size_t(L);
+    pl.prod_bytes = pl.scan ? slots * H * kProdBytes : 0;
     pl.off_prod = off; off = up256(off + pl.prod_bytes);
     pl.total = off;
     return pl;
@@ -1727,9 +1972,12 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
                      int dtype, float scale, int l2norm, void* ws, size_t ws_bytes, cudaStream_t stream,
                      const char** why, int scalar_gate, int out_f32) {
     const int out_dtype = (dtype == KDA_FP32 || out_f32) ? KDA_FP32 : KDA_BF16;
-    const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
+    ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, cu != nullptr, device_sm_count());
     // A workspace of kda_chunk_fwd_workspace() bytes holds the exported chunk products of
     // segmented calls; one of only total_min bytes runs the same schedule recomputing them.
+    // Below a balanced plan's total_min the call runs unsegmented.
+    if (pl.balanced && ws_bytes < pl.total_min)
+        pl = make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, true, device_sm_count(), false);
     const bool products = pl.scan && ws_bytes >= pl.total;
     if (ws_bytes < pl.total_min || (pl.total_min > 0 && ws == nullptr)) {
         *why = "workspace smaller than kda_chunk_fwd_workspace()";
@@ -1785,13 +2033,32 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     cudaEvent_t* ev = g_trace_events;
     if (ev) trace_record(ev[0], stream);
     int* seq_first = pl.scan ? reinterpret_cast<int*>(w + pl.off_first) : nullptr;
-    plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0, seq_first);
+    int* order1 = pl.balanced ? reinterpret_cast<int*>(w + pl.off_order1) : nullptr;
+    int* order2 = pl.balanced ? reinterpret_cast<int*>(w + pl.off_order2) : nullptr;
+    if (pl.balanced) {
+        // per-chunk costs of the three passes, measured at d = 128 on B200 (the output
+        // passes a little dearer with an fp32 o).  The later segments' output passes
+        // are costed as reading back exported products even when the workspace has
+        // no room for them: the cuts, and so the results, do not depend on its size.
+        BalCost cost;
+        const bool f32 = out_dtype == KDA_FP32;
+        cost.whole = f32 ? 14.7f : 13.4f;
+        cost.map = 16.0f;
+        cost.item = 20.0f;
+        cost.light = f32 ? 6.4f : 4.8f;
+        cost.litem = f32 ? 13.0f : 10.0f;
+        cost.comb = 8.45f;
+        cost.seg = 20.0f;
+        plan_balanced_kernel<<<1, 32 * kBalCands, 0, stream>>>(cu, pl.N, H, device_sm_count(), cost, pl.max_items,
+                                                                items, n_items, seq_first, order1, order2);
+    } else {
+        plan_kernel<<<1, 1024, 0, stream>>>(cu, pl.N, T, pl.L, items, n_items, pl.max_items, pl.L0, seq_first);
+    }
     if (ev) trace_record(ev[1], stream);
 
     ChunkArgs a{};
     a.beta = beta;
     a.prod = products ? w + pl.off_prod : nullptr;
-    a.prodL = pl.L;
     a.gs = scalar_gate ? g : nullptr;
     a.init_state = init;
     a.final_state = fin;
@@ -1801,6 +2068,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     a.segN = reinterpret_cast<float*>(w + pl.off_segN);
     a.segX = reinterpret_cast<float*>(w + pl.off_segX);
     a.segS = reinterpret_cast<float*>(w + pl.off_segS);
+    a.order = order1;
+    a.n_order = n_items;
+    a.seg0_whole = pl.balanced ? 1 : 0;
     a.H = H;
     a.scale = scale;
     const dim3 grid(unsigned(pl.max_items), unsigned(H));
@@ -1814,9 +2084,14 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         if (ev) trace_record(ev[2], stream);
         if (!set_smem_attr(combine_kernel, kCombSmem)) return KDA_ERR_CUDA;
         combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), kCombThreads, kCombSmem, stream>>>(
-            items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H);
+            items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H,
+            pl.balanced ? 1 : 0);
         if (ev) trace_record(ev[3], stream);
-        const int r2 = launch_phase_for<2>(out_dtype, scalar_gate, grid, mq, mk, mv, mg, mo, a, stream);
+        ChunkArgs a2 = a;  // a balanced plan launches only the segments g >= 1, longest first
+        a2.order = order2;
+        a2.n_order = n_items + 1;
+        const dim3 grid2 = pl.balanced ? dim3(unsigned(pl.max_items > pl.N ? pl.max_items - pl.N : 1), unsigned(H)) : grid;
+        const int r2 = launch_phase_for<2>(out_dtype, scalar_gate, grid2, mq, mk, mv, mg, mo, a2, stream);
         if (r2 != KDA_OK) return r2;
     }
     if (ev) trace_record(ev[4], stream);
@@ -1849,18 +2124,45 @@ extern "C" int kda_debug_warp_cycles(unsigned long long* out, int reset) {
 
 int chunk_segment_tokens(int B, int T, int H, int num_seqs, int* middle) {
     const ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count());
+    if (pl.balanced) {  // cut per sequence on the device
+        if (middle) *middle = -1;
+        return -1;
+    }
     if (middle) *middle = pl.scan ? pl.L * kC : 0;
     return pl.scan ? pl.L0 * kC : 0;
+}
+
+// The segment table a call with these sizes left in its workspace (it sits at the
+// workspace's start, so dtype and l2norm do not move it).
+int chunk_plan_items(const void* ws, int B, int T, int H, int num_seqs, int* rows, int max_rows) {
+    ChunkPlan pl = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count());
+    const ChunkPlan flat = make_chunk_plan(B, T, H, num_seqs, KDA_BF16, 0, num_seqs > 0, device_sm_count(), false);
+    if (flat.max_items > pl.max_items) pl.max_items = flat.max_items;  // either may have run
+    const uint8_t* w = static_cast<const uint8_t*>(ws);
+    int n = 0;
+    if (cudaMemcpy(&n, w + pl.off_count, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+    if (n < 0 || n > pl.max_items) return -1;
+    const int k = n < max_rows ? n : max_rows;
+    for (int i = 0; i < k; ++i) {
+        SegItem it;
+        if (cudaMemcpy(&it, w + pl.off_items + sizeof(SegItem) * size_t(i), sizeof(SegItem), cudaMemcpyDeviceToHost) !=
+            cudaSuccess)
+            return -1;
+        const int r[5] = {it.seq, it.tok_begin, it.tok_end, it.g, it.G};
+        for (int j = 0; j < 5; ++j) rows[5 * i + j] = r[j];
+    }
+    return n;
 }
 
 size_t chunk_workspace_bytes(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
     return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total;
 }
 
-// The smallest workspace kda_chunk_fwd accepts (the segmented schedule then recomputes
-// the chunk products in its output pass instead of reading them back).
+// The smallest workspace kda_chunk_fwd accepts (a uniform segmented schedule then
+// recomputes the chunk products in its output pass instead of reading them back; a
+// call that would take the balanced plan runs unsegmented).
 size_t chunk_workspace_bytes_min(int B, int T, int H, int num_seqs, int dtype, int l2norm) {
-    return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count()).total_min;
+    return make_chunk_plan(B, T, H, num_seqs, dtype, l2norm, num_seqs > 0, device_sm_count(), false).total_min;
 }
 
 }  // namespace kda

@@ -147,8 +147,24 @@ int kda_set_trace_events(void *events, int n_events);
  * (the last one holds the rest) in *middle_tokens when that is not NULL.  A
  * segmented call runs the segments' maps in one launch, then the combine pass,
  * then the segments' outputs in a second launch.
+ * -1 (and -1 in *middle_tokens) when the cuts depend on the sequence lengths:
+ * packed calls (cu_seqlens) with num_seqs <= 64 whose (sequence, head) pairs
+ * outnumber a third of the SMs and whose total length exceeds 16 chunks.  Their
+ * plan, made on the device from cu_seqlens, cuts each sequence at a common
+ * target length chosen to balance the SMs (short sequences stay whole);
+ * segment 0 then runs its output in the first launch, from the initial state,
+ * and the later segments run their maps there and their outputs in the second.
+ * kda_chunk_fwd_plan_items reports the cuts after a call.
  * Informational (profiling); it never changes what is computed. */
 int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int *middle_tokens);
+
+/* The segment table that the last kda_chunk_fwd or kda_gdn_chunk_fwd call with
+ * these sizes left at the start of `workspace`: copies up to max_rows rows of
+ * five ints (sequence, first token, end token, segment index g, segment count
+ * G) into the host array `rows` and returns the number of segments, or -1 on a
+ * CUDA error.  Synchronous (it waits for the device).  Informational: tests and
+ * profiling. */
+int kda_chunk_fwd_plan_items(const void *workspace, int B, int T, int H, int num_seqs, int *rows, int max_rows);
 
 /* Workspace bytes for a kda_chunk_fwd call with the same B, T, H, num_seqs
  * (0 = dense), dtype and l2norm_qk, on the current device. */
@@ -159,7 +175,12 @@ size_t kda_chunk_fwd_workspace(int B, int T, int H, int num_seqs, int dtype, int
  * each segment map pass's per-chunk products (about 66 KB per chunk and head,
  * e.g. ~1.2 GB at B=1 H=16 T=65536) and its output pass reads them back instead
  * of recomputing them; with less (but at least this many) bytes it recomputes
- * them.  Both give bit-identical results; the first is faster. */
+ * them.  Both give bit-identical results; the first is faster.
+ * Calls that take the balanced plan (kda_chunk_fwd_segment_tokens() == -1) also
+ * need per-segment states, up to (num_seqs + ceil((T/64 + num_seqs) / 16)) x H
+ * x 192 KiB.  With a workspace smaller than that (but at least this many bytes)
+ * they run unsegmented, one CTA per (sequence, head): slower, and equal to the
+ * segmented results only up to rounding. */
 size_t kda_chunk_fwd_workspace_min(int B, int T, int H, int num_seqs, int dtype, int l2norm_qk);
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -50,7 +50,9 @@ def test_segment_plan_on_148_sms(kda):
     """Host-side plan (no device here: the library assumes a B200's 148 SMs).  With
     P = sequences x heads <= 148/3 pairs, each sequence is cut into G = 148 // P equal
     segments of L = ceil((chunks + 1) / G) chunks (the last holds the rest): one CTA per
-    segment and pair in each phase.  With more pairs every (sequence, head) runs whole."""
+    segment and pair in each phase.  With more pairs every (sequence, head) of a dense
+    call runs whole; packed calls of at most 64 sequences longer than 16 chunks in all
+    are cut on the device (the balanced plan), which the query reports as -1."""
     # B=1 H=16 T=65536: 1024 chunks, G = 9, L = ceil(1025 / 9) = 114 chunks
     assert kda.chunk_fwd_segments(1, 65536, 16) == (114 * 64, 114 * 64)
     # T=16384: 256 chunks, L = ceil(257 / 9) = 29
@@ -60,8 +62,20 @@ def test_segment_plan_on_148_sms(kda):
     # 256 or 50 pairs (> 148 / 3): no segment scan
     assert kda.chunk_fwd_segments(16, 4096, 16) == (0, 0)
     assert kda.chunk_fwd_segments(1, 65536, 50) == (0, 0)
-    # packed sequences count as separate pairs: 8 sequences x 16 heads = 128 pairs
-    assert kda.chunk_fwd_segments(1, 65536, 16, 8) == (0, 0)
+    # packed sequences count as separate pairs: 8 sequences x 16 heads = 128 pairs, so
+    # the plan is made on the device from the lengths (balanced)
+    assert kda.chunk_fwd_segments(1, 65536, 16, 8) == (-1, -1)
+    # ... unless they are too many (> 64) or too short (16 chunks in all) to cut
+    assert kda.chunk_fwd_segments(1, 65536, 16, 65) == (0, 0)
+    assert kda.chunk_fwd_segments(1, 1024, 16, 8) == (0, 0)
+    assert kda.chunk_fwd_segments(1, 1025, 16, 8) == (-1, -1)
+    # its workspace holds one product image per chunk of the call and head, and the
+    # per-segment states of at most N + ceil((chunks + N) / 16) segments; the minimal
+    # workspace (the call then runs unsegmented) holds neither
+    full = kda.lib().kda_chunk_fwd_workspace(1, 65536, 16, 8, 0, 0)
+    small = kda.lib().kda_chunk_fwd_workspace_min(1, 65536, 16, 8, 0, 0)
+    assert full - small >= (1024 + 8) * 16 * 67584 + 3 * (8 + 65) * 16 * 128 * 128 * 4
+    assert small < 4096
     # too short to pay for the map pass: fewer than 3 segments' worth of chunks
     assert kda.chunk_fwd_segments(1, 64, 49) == (0, 0)
     # the product images only fit the full workspace; the minimal one runs the same plan

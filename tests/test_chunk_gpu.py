@@ -133,6 +133,64 @@ def test_varlen_mixes_whole_and_segmented_sequences(kda):
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
 
 
+# 8 packed sequences of 100 ... 5000 tokens (2 to 79 chunks) x 16 heads: 128 pairs,
+# too many for the uniform segment plan, so the device cuts the lengths itself.
+BALANCED_CU = [0, 100, 5100, 5164, 7164, 7165, 11165, 11900, 12000]
+
+
+def test_balanced_plan_cuts_long_packed_sequences(kda):
+    """The device plan keeps the short sequences whole and cuts the long ones at a
+    common target length: segment 0 runs its output in the first launch from the
+    initial state, the later segments a map there and their output in the second
+    launch, and sequences of three or more segments chain their maps through the
+    combine pass.  Parity against the oracle on four heads; the same bits whether
+    the later segments read back the exported chunk products (the full workspace)
+    or recompute them (any smaller workspace that still holds the per-segment
+    states); the minimal workspace runs unsegmented, within rounding."""
+    cu, H = BALANCED_CU, 16
+    T, nseq = cu[-1], len(cu) - 1
+    assert kda.chunk_fwd_segments(1, T, H, nseq) == (-1, -1)
+    inp = synth.op_inputs(B=nseq, H=H, T=T, s0_std=0.02, seed=31, cu_seqlens=cu)
+    eo, es = run_both(kda, inp, heads=[0, 5, 10, 15])
+    assert eo < TOL and es < TOL, (eo, es)
+    d = [inp[n].cuda() for n in ("q", "k", "v", "g", "beta")]
+    cu_d, s0 = inp["cu_seqlens"].cuda(), inp["s0"].cuda()
+    lib = kda.lib()
+    full = lib.kda_chunk_fwd_workspace(1, T, H, nseq, 0, 0)
+    small = lib.kda_chunk_fwd_workspace_min(1, T, H, nseq, 0, 0)
+    assert small < full - 256
+    res, plans = [], []
+    for nbytes in (full, full - 256, small):
+        ws = torch.empty(nbytes, device="cuda", dtype=torch.uint8)
+        res.append(kda.chunk_fwd(*d, initial_state=s0, cu_seqlens=cu_d, workspace=ws))
+        plans.append(kda.chunk_fwd_plan(ws, 1, T, H, nseq))
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert plans[0] == plans[1] and len(plans[2]) == nseq  # the minimal workspace: one item per sequence
+    for a, b in zip(res[0], res[2]):
+        assert rel_l2(f64(a), f64(b)) < 5e-3
+    plan = plans[0]
+    # the segments tile every sequence in order, on chunk boundaries
+    for n in range(nseq):
+        segs = [r for r in plan if r[0] == n]
+        assert segs[0][1] == cu[n] and segs[-1][2] == cu[n + 1]
+        assert [r[3] for r in segs] == list(range(len(segs))) and all(r[4] == len(segs) for r in segs)
+        for a, b in zip(segs, segs[1:]):
+            assert a[2] == b[1] and (b[1] - cu[n]) % 64 == 0 and b[1] < b[2]
+    G = {r[0]: r[4] for r in plan}
+    print("segments per sequence:", [G[n] for n in range(nseq)])
+    assert G[1] >= 3 and G[0] == 1 and G[4] == 1  # the 5000-token one chains; 100 and 1 token stay whole
+
+
+def test_balanced_plan_with_empty_sequences_and_no_initial_state(kda):
+    cu = [0, 0, 3000, 3000, 3001, 4500, 4500, 9000, 9100]
+    inp = synth.op_inputs(B=len(cu) - 1, H=16, T=cu[-1], s0_std=None, seed=32, cu_seqlens=cu)
+    assert kda.chunk_fwd_segments(1, cu[-1], 16, len(cu) - 1) == (-1, -1)
+    eo, es = run_both(kda, inp, heads=[3, 12])
+    assert eo < TOL and es < TOL, (eo, es)
+
+
 def test_final_state_only_and_zero_state(kda):
     inp = synth.op_inputs(B=2, H=2, T=100, s0_std=None, seed=14)
     eo, es = run_both(kda, inp)

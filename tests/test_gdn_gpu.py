@@ -127,3 +127,13 @@ def test_gdn_prefill_64k_sampled_heads(kda):
     inp = gdn_inputs(**{**synth.prefill_sweep(65536), "device": "cuda"})
     eo, es = run_both(kda, inp, heads=[3, 7, 12, 14])
     assert eo < TOL and es < TOL, (eo, es)
+
+
+def test_balanced_plan_packed_sequences(kda):
+    """Packed sequences with 128 (sequence, head) pairs take the device-made
+    balanced plan; the scalar-gate kernels share it."""
+    cu = [0, 100, 5100, 5164, 7164, 7165, 11165, 11900, 12000]
+    assert kda.chunk_fwd_segments(1, cu[-1], 16, len(cu) - 1) == (-1, -1)
+    inp = gdn_inputs(B=len(cu) - 1, H=16, T=cu[-1], s0_std=0.02, seed=33, cu_seqlens=cu)
+    eo, es = run_both(kda, inp, heads=[1, 14])
+    assert eo < TOL and es < TOL, (eo, es)
