@@ -215,7 +215,10 @@ constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 // channel shares it, so the decay factors are per row instead of per element.
 constexpr int kThreads = 512;  // 16 warps; 4 threads per TMEM lane (one per column quarter)
 
-template <bool kSummary, typename OutT, bool kScalarGate>
+// kChain = false (summary only): the last segment's map in a balanced plan, which
+// runs only to export its chunk products (they do not depend on the state) and so
+// skips the state and transition chains, which no later pass reads.
+template <bool kSummary, typename OutT, bool kScalarGate, bool kChain = true>
 __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                            const CUtensorMap& tm_g, const CUtensorMap& tm_o, const ChunkArgs& p,
                                            const SegItem it, const int item_id, const int h) {
@@ -281,6 +284,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 
     const int t_begin = it.tok_begin, t_end = it.tok_end;
     const int nchunks = (t_end - t_begin + kC - 1) / kC;
+    static_assert(kChain || kSummary, "only a map pass may skip the chains");
+    constexpr bool chain = kChain;
 
     auto issue_qkg = [&](int c) -> bool {  // false: skipped by the failure-test hook
         if (c == c_skip_chunk_load) return false;
@@ -640,7 +645,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) tmem_st16(tbase + tcol + lane_off + part * 32 + cb * 16, x + cb * 16);
             };
-            frame(TM_S, OFF_ST, OFF_ST + 16384);
+            if (chain) frame(TM_S, OFF_ST, OFF_ST + 16384);
             if (!kSummary) {  // O^T starts at zero: the merged [U~|O] MMA below accumulates into both halves
                 float z[16];
 #pragma unroll
@@ -752,7 +757,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         tc_fence_after();
         KDA_WMARK(1);
         KDA_STAGE(3);
-        if (kSummary && warp >= 4) {
+        if (kSummary && chain && warp >= 4) {
             // X' = X e^{mp} as bf16 pairs into the [A;P] columns (read out by now): the A operand
             // of the U_X~ MMA; TMEM X <- X e^{mk}.  Warps 4..15 do it while warps 0..3 run the
             // diagonal UT solves: the three warps of a TMEM lane quadrant take key columns
@@ -968,7 +973,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 
         KDA_STAGE(9);
         // ===== U~^T = U^T - S'^T W^T ;  O^T = S'^T Qp  (or U_X~^T = -X'^T W^T) =====
-        if (tid == 0) {
+        if (chain && tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -998,8 +1003,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             e_rows(0, true);
         }
         KDA_STAGE(16);
-        ok = mbar_wait(&bars[2], ph_mma, 5);
-        ph_mma ^= 1;
+        if (chain) {
+            ok = mbar_wait(&bars[2], ph_mma, 5);
+            ph_mma ^= 1;
+        }
         tc_fence_after();
         // the exports have read Qp (rewritten next) and T beta + P (U_X~^T goes over them)
         if (img && tid == kExporter) bulk_wait_read0();
@@ -1017,8 +1024,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                                  pack_bf16x2(u[q4 * 8 + 0], u[q4 * 8 + 1]), pack_bf16x2(u[q4 * 8 + 2], u[q4 * 8 + 3]),
                                  pack_bf16x2(u[q4 * 8 + 4], u[q4 * 8 + 5]), pack_bf16x2(u[q4 * 8 + 6], u[q4 * 8 + 7]));
             };
-            spill(TM_U, OFF_UT);
-            if (kSummary) spill(TM_O, UXT);
+            if (chain) spill(TM_U, OFF_UT);
+            if (kSummary && chain) spill(TM_O, UXT);
         }
         fence_async_smem();
         tc_fence_before();
@@ -1026,7 +1033,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
 
         KDA_STAGE(11);
         // ===== O^T += U~^T P^T ;  S^T += U~^T Km  (X^T += U_X~^T Km) =====
-        if (tid == 0) {
+        if (chain && tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
@@ -1046,8 +1053,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             e_put_kq(1);
         }
         KDA_STAGE(18);
-        ok = mbar_wait(&bars[2], ph_mma, 6);
-        ph_mma ^= 1;
+        if (chain) {
+            ok = mbar_wait(&bars[2], ph_mma, 6);
+            ph_mma ^= 1;
+        }
         tc_fence_after();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         KDA_STAGE(12);
@@ -1102,8 +1111,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
         float* dstS = nullptr;
         float* dstX = nullptr;
         if (kSummary) {
-            dstS = p.segN + (size_t(item_id) * H + h) * (kD * kD);
-            dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
+            if (chain) {
+                dstS = p.segN + (size_t(item_id) * H + h) * (kD * kD);
+                dstX = p.segX + (size_t(item_id) * H + h) * (kD * kD);
+            }
         } else if (it.g == it.G - 1) {
             if (p.final_state) dstS = p.final_state + (size_t(it.seq) * H + h) * (kD * kD);
         } else if (p.seg0_whole && it.g == 0 && item_id + 1 < *p.n_items) {  // the start state of segment 1
@@ -1428,8 +1439,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const SegItem it = p.items[item];
     if (it.G == 1 || (p.seg0_whole && it.g == 0))
         chunk_body<false, OutT, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
-    else if (it.g < it.G - 1 || p.prod)
+    else if (it.g < it.G - 1 || (p.prod && !p.seg0_whole))
         chunk_body<true, __nv_bfloat16, kScalarGate>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
+    else if (p.prod)  // a balanced plan's last segment: chunk products only.  (A uniform plan's segments are
+                      // equal, so its phase 1 lasts as long as a full map whatever the last one does; it keeps
+                      // one code path for every CTA.)
+        chunk_body<true, __nv_bfloat16, kScalarGate, false>(tm_q, tm_k, tm_v, tm_g, tm_o, p, it, item, h);
 }
 
 // Phase 2: the outputs of every segment of a segmented sequence from its start
@@ -1519,10 +1534,12 @@ constexpr int kBalMinChunks = 16;  // shortest target segment length
 constexpr int kBalCands = 16;      // target lengths tried: ceil(longest / (w + 1)), w < 16
 
 // Costs that the plan weighs, in thousands of SM cycles on B200 (fitted to the
-// phase times of 24 plans over three length mixes, all SMs busy).
+// phase times of forced target lengths 16-128 over three length mixes of 65536
+// packed tokens, H=16, bf16 and fp32 o, all SMs busy).
 struct BalCost {
     float whole;  // per chunk of an output pass from a known start state (segment 0, whole sequences)
     float map;    // per chunk of a map pass
+    float prod;   // per chunk of the last segment's map pass (chunk products only, no chains)
     float item;   // per phase-1 CTA: TMEM and barriers, the start state in, the end state out
     float light;  // per chunk of a later segment's output pass
     float litem;  // per phase-2 CTA
@@ -1591,7 +1608,8 @@ __global__ void __launch_bounds__(32 * kBalCands) plan_balanced_kernel(const int
             max1 = fmaxf(max1, c0);
             for (int g = 1; g < G; ++g) {
                 const int len = min(lm, nch - l0 - (g - 1) * lm);
-                const float cm = float(len) * cost.map + cost.item, cl = float(len) * cost.light + cost.litem;
+                const float cm = float(len) * (g == G - 1 ? cost.prod : cost.map) + cost.item;
+                const float cl = float(len) * cost.light + cost.litem;
                 sum1 += cm;
                 max1 = fmaxf(max1, cm);
                 sum2 += cl;
@@ -1669,7 +1687,7 @@ __global__ void __launch_bounds__(32 * kBalCands) plan_balanced_kernel(const int
             s.slot = sb / kC + tid + c0;  // distinct for every chunk of every sequence
             s.pad1 = 0;
             items[off + g] = s;
-            s_k1[off + g] = float(c1 - c0) * (g == 0 ? cost.whole : cost.map);
+            s_k1[off + g] = float(c1 - c0) * (g == 0 ? cost.whole : (g == G - 1 ? cost.prod : cost.map));
             s_k2[off + g] = g == 0 ? -1.f : float(c1 - c0);
         }
     }
@@ -2043,7 +2061,8 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
         BalCost cost;
         const bool f32 = out_dtype == KDA_FP32;
         cost.whole = f32 ? 14.7f : 13.4f;
-        cost.map = 16.0f;
+        cost.map = 17.0f;
+        cost.prod = 13.0f;
         cost.item = 20.0f;
         cost.light = f32 ? 6.4f : 4.8f;
         cost.litem = f32 ? 13.0f : 10.0f;
