@@ -144,6 +144,11 @@ struct ChunkArgs {
     float scale;
 };
 
+// Column swizzle of the segment maps' X^T rows in global memory (and, by a linear
+// copy, in the combine pass's shared memory): column k of row k' sits at k ^ this.
+// Rows k' .. k'+3 of one MMA fragment then spread one column over 4 x 8 banks.
+__device__ __forceinline__ int xt_swizzle(int kp) { return (kp & 3) << 3; }
+
 // fp32 -> tf32 operand, rounded to nearest (ties away from zero) on the integer
 // pipe: add half an ulp of the 10-bit mantissa to the magnitude bits, then drop
 // the 13 low bits.  Finite inputs only.
@@ -1133,19 +1138,21 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
             }
         };
         if (dstS) store(TM_S, dstS);
-        if (dstX) {  // X stored transposed, [k'][k] (TMEM lane k' owns a contiguous row), for the combine pass
+        if (dstX) {  // X stored transposed, [k'][k] (TMEM lane k' owns a row), for the combine pass, with
+                     // column k of row k' at k ^ xt_swizzle(k') (see the combine pass)
+            float* row = dstX + size_t(vrow) * kD;
+            const int sw = xt_swizzle(vrow);
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
                 const int k0 = part * 32 + cb * 16;
                 float x[16];
                 tmem_ld16(tbase + TM_X + lane_off + k0, x);
                 tmem_wait_ld();
-                float4* d4 = reinterpret_cast<float4*>(dstX + size_t(vrow) * kD + k0);
 #pragma unroll
                 for (int j = 0; j < 16; j += 4)
-                    d4[j >> 2] = make_float4(x[j] * sPost[last * 128 + k0 + j], x[j + 1] * sPost[last * 128 + k0 + j + 1],
-                                             x[j + 2] * sPost[last * 128 + k0 + j + 2],
-                                             x[j + 3] * sPost[last * 128 + k0 + j + 3]);
+                    *reinterpret_cast<float4*>(row + ((k0 + j) ^ sw)) =
+                        make_float4(x[j] * sPost[last * 128 + k0 + j], x[j + 1] * sPost[last * 128 + k0 + j + 1],
+                                    x[j + 2] * sPost[last * 128 + k0 + j + 2], x[j + 3] * sPost[last * 128 + k0 + j + 3]);
             }
         }
     } else {
@@ -1712,14 +1719,25 @@ __global__ void __launch_bounds__(32 * kBalCands) plan_balanced_kernel(const int
 // Chains the segment maps of one (sequence, head, 16-column slice):
 // S_{g+1} = X_g S_g + N_g, written as the start state of segment g+1 (segment 0
 // gets the initial state).  With s0 = 1 (balanced plans) phase 1 has already
-// written S_1, the end state of segment 0's output pass, and the chain starts there.  X_g^T (64 KB, written transposed by the summary
-// pass) streams into shared memory with 1-D bulk copies, double-buffered.  Two
-// halves of 256 threads each sum over half of the key dimension, a thread owning
-// a 2 x 4 tile of the slice; the halves' sums meet in shared memory.
+// written S_1, the end state of segment 0's output pass, and the chain starts there.
+// X_g^T (64 KB, written transposed and column-swizzled by the summary pass) streams
+// into shared memory with one 1-D bulk copy per step, double-buffered.  Each of the 8
+// warps owns 16 rows of the 128 x 16 product and runs them on tf32 warp MMAs split
+// three ways (hi*hi + hi*lo + lo*hi, with x = hi + lo both tf32): fp32-level
+// accuracy at tensor-core latency.  The swizzle makes the A-fragment loads (4 rows
+// of X^T x 8 columns per warp) hit 32 distinct banks; the slice of S is
+// double-buffered with rows padded to 24 floats (conflict-free B fragments), so one
+// barrier per step orders both buffers; N_{g+1}'s slice is loaded a step ahead.
 constexpr int kCombCols = 16;
-constexpr int kCombThreads = 512;  // two halves of 256, each summing over half of the key dimension
-constexpr uint32_t kCombSmem = 2 * 65536 + kD * kCombCols * 4 + 256 * 8 * 4 + 64;
+constexpr int kCombThreads = 256;  // 8 warps, one 16-row tile of the 128 x 16 slice each
+constexpr int kCombSs = 24;        // S slice row stride in shared memory (floats)
+constexpr uint32_t kCombSmem = 2 * 65536 + 2 * kD * kCombSs * 4 + 64;
 
+// x = hi + lo, both exactly representable in tf32 (hi rounded to nearest).
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = f32_to_tf32(x);
+    lo = f32_to_tf32(x - __uint_as_float(hi));
+}
 
 __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem* items, const int* n_items,
                                                                   const int* seq_first, int N, const float* init,
@@ -1732,13 +1750,12 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem*
     const SegItem it = items[item];
     if (it.g != 0 || it.G < 2 + s0) return;
     extern __shared__ __align__(128) uint8_t csm[];
-    float* sX = reinterpret_cast<float*>(csm);                       // [2][128 k'][128 k]
-    float* sS = reinterpret_cast<float*>(csm + 2 * 65536);           // [128 k][16 j]
-    float* sR = sS + kD * kCombCols;                                 // [256][8] the upper half's partial sums
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sR + 256 * 8);       // [2]
-    const int tid = threadIdx.x, half = tid >> 8, t = tid & 255;
-    const int k0 = (t >> 2) * 2, j0 = (t & 3) * 4;  // rows k0, k0+1; cols j0..j0+3 of the slice
-    const int kp0 = half * (kD / 2);                 // this half's key range [kp0, kp0 + 64)
+    float* sX = reinterpret_cast<float*>(csm);                            // [2][128 k'][128 k]: X_g^T, swizzled
+    float* sS = sX + 2 * kD * kD;                                         // [2][128 k][kCombSs]: S_g's slice
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sS + 2 * kD * kCombSs);  // [2]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int m0 = warp * 16;  // this warp's rows k
     const int c0 = kCombCols * z;
     const size_t hs = size_t(h) * (kD * kD);
     if (tid == 0) {
@@ -1759,10 +1776,28 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem*
                            : (init ? init + size_t(it.seq) * H * (kD * kD) + hs : nullptr);
     for (int e = tid; e < kD * kCombCols; e += kCombThreads) {
         const int kk = e / kCombCols, jj = e % kCombCols;
-        sS[e] = s_in ? s_in[size_t(kk) * kD + c0 + jj] : 0.f;
+        sS[kk * kCombSs + jj] = s_in ? s_in[size_t(kk) * kD + c0 + jj] : 0.f;
     }
-    __syncthreads();
     const int steps = it.G - 1 - s0;
+    // this thread's accumulators: rows m0 + gq (+8), columns 8 nt + 2 tq (+1), nt = 0, 1
+    auto load_n = [&](int g, float* v) {
+        const float* b = segN + size_t(item + g) * H * (kD * kD) + hs + size_t(m0 + gq) * kD + c0 + 2 * tq;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float2 a = *reinterpret_cast<const float2*>(b + 8 * nt);
+            const float2 c = *reinterpret_cast<const float2*>(b + 8 * kD + 8 * nt);
+            v[nt * 4 + 0] = a.x;
+            v[nt * 4 + 1] = a.y;
+            v[nt * 4 + 2] = c.x;
+            v[nt * 4 + 3] = c.y;
+        }
+    };
+    float nxt[8];
+    load_n(s0, nxt);
+    __syncthreads();
+    // A-fragment columns: k = m0 + gq (+8), swizzled by row k' = kp + tq (+4), whose low two bits are tq
+    const int sw = tq << 3;
+    const int ca = (m0 + gq) ^ sw, cb = (m0 + gq + 8) ^ sw;
     bool ok = true;
     int fetched = 1, j = 0;  // fetches issued (thread 0) and the step being consumed
     for (; j < steps; ++j) {
@@ -1771,52 +1806,53 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem*
             fetch(j + 1);
             fetched = j + 2;
         }
-        const size_t base = size_t(item + g) * H * (kD * kD) + hs;
-        float acc[2][4];
+        float acc[8], x1[8], x2[8];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {  // the lower half starts from N_g's slice (requested before the wait)
-            float4 n4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (half == 0) n4 = *reinterpret_cast<const float4*>(segN + base + size_t(k0 + r) * kD + c0 + j0);
-            acc[r][0] = n4.x; acc[r][1] = n4.y; acc[r][2] = n4.z; acc[r][3] = n4.w;
+        for (int e = 0; e < 8; ++e) {
+            acc[e] = nxt[e];
+            x1[e] = x2[e] = 0.f;
         }
+        if (j + 1 < steps) load_n(g + 1, nxt);
         ok = mbar_wait(&bar[j & 1], uint32_t((j >> 1) & 1), 8);
         if (__syncthreads_or(!ok)) break;
-        const float* X = sX + (j & 1) * kD * kD;
-#pragma unroll 1
-        for (int kb = kp0; kb < kp0 + kD / 2; kb += 8) {  // acc[k][j] += Xt[kp][k] S[kp][j]
-            float2 xv[8];  // 8 key steps' operands requested before their FMAs (hides the load latency)
-            float4 sv[8];
+        const float* X = sX + (j & 1) * kD * kD;  // X^T: row k', column k (swizzled)
+        const float* S = sS + (j & 1) * kD * kCombSs;
+#pragma unroll 2
+        for (int kp = 0; kp < kD; kp += 8) {
+            // A (16 x 8): A[m][kk] = X^T[kp + kk][m0 + m];  B (8 x 8) per column tile: S[kp + kk][8 nt + n]
+            const float* r0 = X + (kp + tq) * kD;
+            const float* r4 = r0 + 4 * kD;
+            uint32_t ah[4], al[4];
+            split_tf32(r0[ca], ah[0], al[0]);
+            split_tf32(r0[cb], ah[1], al[1]);
+            split_tf32(r4[ca], ah[2], al[2]);
+            split_tf32(r4[cb], ah[3], al[3]);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                xv[u] = *reinterpret_cast<const float2*>(X + (kb + u) * kD + k0);
-                sv[u] = *reinterpret_cast<const float4*>(sS + (kb + u) * kCombCols + j0);
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bh[2], bl[2];
+                split_tf32(S[(kp + tq) * kCombSs + 8 * nt + gq], bh[0], bl[0]);
+                split_tf32(S[(kp + tq + 4) * kCombSs + 8 * nt + gq], bh[1], bl[1]);
+                mma_tf32_16x8x8(acc + 4 * nt, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                mma_tf32_16x8x8(x1 + 4 * nt, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                mma_tf32_16x8x8(x2 + 4 * nt, al[0], al[1], al[2], al[3], bh[0], bh[1]);
             }
+        }
+        float* Sn = sS + ((j + 1) & 1) * kD * kCombSs;
+        float* out = segS + size_t(item + g + 1) * H * (kD * kD) + hs;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                acc[0][0] += xv[u].x * sv[u].x; acc[0][1] += xv[u].x * sv[u].y;
-                acc[0][2] += xv[u].x * sv[u].z; acc[0][3] += xv[u].x * sv[u].w;
-                acc[1][0] += xv[u].y * sv[u].x; acc[1][1] += xv[u].y * sv[u].y;
-                acc[1][2] += xv[u].y * sv[u].z; acc[1][3] += xv[u].y * sv[u].w;
-            }
+        for (int nt = 0; nt < 2; ++nt) {
+            const int r = m0 + gq, cc = 8 * nt + 2 * tq;
+            const float* a = acc + 4 * nt;
+            const float* p1 = x1 + 4 * nt;
+            const float* p2 = x2 + 4 * nt;
+            const float2 v0 = make_float2(a[0] + (p1[0] + p2[0]), a[1] + (p1[1] + p2[1]));
+            const float2 v1 = make_float2(a[2] + (p1[2] + p2[2]), a[3] + (p1[3] + p2[3]));
+            *reinterpret_cast<float2*>(Sn + r * kCombSs + cc) = v0;
+            *reinterpret_cast<float2*>(Sn + (r + 8) * kCombSs + cc) = v1;
+            *reinterpret_cast<float2*>(out + size_t(r) * kD + c0 + cc) = v0;
+            *reinterpret_cast<float2*>(out + size_t(r + 8) * kD + c0 + cc) = v1;
         }
-        if (half == 1) {
-            float4* r4 = reinterpret_cast<float4*>(sR + t * 8);
-            r4[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-            r4[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-        }
-        __syncthreads();  // every thread has read sS and this X buffer; the upper half's sums are in sR
-        if (half == 0) {
-            const float4* r4 = reinterpret_cast<const float4*>(sR + t * 8);
-            const float4 p0 = r4[0], p1 = r4[1];
-            const size_t out = size_t(item + g + 1) * H * (kD * kD) + hs;
-            const float4 v0 = make_float4(acc[0][0] + p0.x, acc[0][1] + p0.y, acc[0][2] + p0.z, acc[0][3] + p0.w);
-            const float4 v1 = make_float4(acc[1][0] + p1.x, acc[1][1] + p1.y, acc[1][2] + p1.z, acc[1][3] + p1.w);
-            *reinterpret_cast<float4*>(sS + k0 * kCombCols + j0) = v0;
-            *reinterpret_cast<float4*>(sS + (k0 + 1) * kCombCols + j0) = v1;
-            *reinterpret_cast<float4*>(segS + out + size_t(k0) * kD + c0 + j0) = v0;
-            *reinterpret_cast<float4*>(segS + out + size_t(k0 + 1) * kD + c0 + j0) = v1;
-        }
-        __syncthreads();
+        __syncthreads();  // every warp has read this X buffer and S buffer; S_{g+1} is complete
     }
     if (tid == 0 && !ok) {  // let copies still in flight land before the shared memory is released
         for (int f = j; f < fetched; ++f) mbar_wait(&bar[f & 1], uint32_t((f >> 1) & 1), 8);
