@@ -369,27 +369,37 @@ def run_ours(args):
     assert kda.device_status() == 0
 
     def timed_steps(fn, traces):
-        """Time args.steps calls of fn with per-call trace events on the launching stream.
-        The calls are captured into one CUDA graph and replayed, so host-side jitter
-        between calls cannot leave the GPU idle; --eager times them as issued."""
+        """Time args.steps calls of fn.  The calls are captured into one CUDA graph and
+        replayed, so host-side jitter between calls cannot leave the GPU idle.  The
+        per-launch breakdown comes from a second graph of the same calls with the
+        library's trace events, replayed after the timed one: an event between two
+        launches keeps the second from starting while the first finishes (the
+        library's programmatic dependent launches), so the timed graph has none.
+        --eager times the traced calls as issued."""
         for tr in traces:  # create the events outside the capture
             for e in tr:
                 e.record(stream)
-        graph, timing = None, "eager: K calls issued back to back"
+        graph, traced, timing = None, None, "eager: K calls issued back to back"
         if not args.eager:
             try:
                 graph = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(graph):
                     for i in range(args.steps):
+                        fn()
+                traced = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(traced):
+                    for i in range(args.steps):
                         kda.set_trace_events(traces[i])
                         fn()
                 kda.set_trace_events(None)
-                graph.replay()  # untimed: uploads the graph
+                graph.replay()  # untimed: uploads the graphs
+                traced.replay()
                 torch.cuda.synchronize()
-                timing = "one CUDA graph of the K calls, replayed once"
+                timing = ("one CUDA graph of the K calls, replayed once; the per-launch times come from a "
+                          "second graph with trace events between the launches")
             except Exception as exc:  # fall back to timing the calls as issued
                 kda.set_trace_events(None)
-                graph = None
+                graph = traced = None
                 torch.cuda.synchronize()
                 print(f"bench: CUDA graph capture failed ({exc}); timing eagerly", file=sys.stderr)
         assert kda.device_status() == 0
@@ -406,6 +416,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         kda.set_trace_events(None)
+        if traced is not None:  # untimed: the per-launch breakdown
+            traced.replay()
+            torch.cuda.synchronize()
         return start.elapsed_time(end) / args.steps, timing
 
     # timed region: K steps
