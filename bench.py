@@ -372,10 +372,9 @@ def run_ours(args):
         """Time args.steps calls of fn.  The calls are captured into one CUDA graph and
         replayed, so host-side jitter between calls cannot leave the GPU idle.  The
         per-launch breakdown comes from a second graph of the same calls with the
-        library's trace events, replayed after the timed one: an event between two
-        launches keeps the second from starting while the first finishes (the
-        library's programmatic dependent launches), so the timed graph has none.
-        --eager times the traced calls as issued."""
+        library's trace events (event nodes between the launches), replayed after the
+        timed one, so that the timed graph holds the calls alone.  --eager times the
+        traced calls as issued."""
         for tr in traces:  # create the events outside the capture
             for e in tr:
                 e.record(stream)

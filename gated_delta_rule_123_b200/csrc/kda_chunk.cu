@@ -1441,8 +1441,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
-    pdl_trigger();  // the combine pass may launch once every CTA here has started
-    pdl_wait();     // the plan has been written
     int item, h;
     if (!cta_item(p, item, h)) return;
     const SegItem it = p.items[item];
@@ -1464,7 +1462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_phase2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                         const __grid_constant__ CUtensorMap tm_o, const ChunkArgs p) {
-    pdl_wait();  // the combine pass (and before it phase 1 and the plan) has completed
     int item, h;
     if (!cta_item(p, item, h)) return;
     const SegItem it = p.items[item];
@@ -1482,7 +1479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Segment 0 of a sequence has L0 chunks, the others L (the last one the rest).
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* cu, int N, int T, int L, SegItem* items,
                                                     int* n_items, int max_items, int L0, int* seq_first) {
-    pdl_trigger();  // phase 1 may launch now; it waits for this grid before reading the plan
     using Scan = cub::BlockScan<int, 1024>;
     __shared__ typename Scan::TempStorage tmp;
     __shared__ int s_base;
@@ -1585,7 +1581,6 @@ __global__ void __launch_bounds__(32 * kBalCands) plan_balanced_kernel(const int
                                                                        BalCost cost, int max_items, SegItem* items,
                                                                        int* counts, int* seq_first, int* order1,
                                                                        int* order2) {
-    pdl_trigger();  // phase 1 may launch now; it waits for this grid before reading the plan
     __shared__ int s_n[kBalMaxSeqs], s_off[kBalMaxSeqs + 1];
     __shared__ unsigned long long s_key[kBalCands];
     __shared__ float s_k1[kBalMaxItems], s_k2[kBalMaxItems];
@@ -1748,8 +1743,6 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const SegItem*
                                                                   const int* seq_first, int N, const float* init,
                                                                   const float* segN, const float* segXt,
                                                                   float* segS, int H, int s0) {
-    pdl_trigger();  // phase 2 may launch once every CTA here has started
-    pdl_wait();     // phase 1's maps (and the plan) are written
     const int n = blockIdx.x, h = blockIdx.y, z = blockIdx.z;  // one CTA per (sequence, head, slice)
     if (n >= N) return;
     const int item = seq_first[n];
@@ -2001,10 +1994,8 @@ static int launch_phase(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk,
                         const CUtensorMap& mg, const CUtensorMap& mo, const ChunkArgs& a, cudaStream_t stream) {
     auto kern = kPhase == 1 ? chunk_phase1_kernel<O, G> : chunk_phase2_kernel<O, G>;
     if (!set_smem_attr(kern, kSmemBytes)) return KDA_ERR_CUDA;
-    // each phase follows the plan or the combine pass in the stream: its launch overlaps their tail
-    return launch_dependent(kern, grid, dim3(kThreads), kSmemBytes, stream, mq, mk, mv, mg, mo, a) == cudaSuccess
-               ? KDA_OK
-               : KDA_ERR_CUDA;
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, a);
+    return KDA_OK;
 }
 
 template <int kPhase>
@@ -2147,14 +2138,9 @@ int launch_chunk_fwd(const void* q, const void* k, const void* v, const float* g
     if (pl.scan) {
         if (ev) trace_record(ev[2], stream);
         if (!set_smem_attr(combine_kernel, kCombSmem)) return KDA_ERR_CUDA;
-        if (launch_dependent(combine_kernel, dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), dim3(kCombThreads),
-                             kCombSmem, stream, static_cast<const SegItem*>(items), static_cast<const int*>(n_items),
-                             static_cast<const int*>(seq_first), pl.N, init, static_cast<const float*>(a.segN),
-                             static_cast<const float*>(a.segX), reinterpret_cast<float*>(w + pl.off_segS), H,
-                             pl.balanced ? 1 : 0) != cudaSuccess) {
-            *why = "combine launch failed";
-            return KDA_ERR_CUDA;
-        }
+        combine_kernel<<<dim3(unsigned(pl.N), unsigned(H), kD / kCombCols), kCombThreads, kCombSmem, stream>>>(
+            items, n_items, seq_first, pl.N, init, a.segN, a.segX, reinterpret_cast<float*>(w + pl.off_segS), H,
+            pl.balanced ? 1 : 0);
         if (ev) trace_record(ev[3], stream);
         ChunkArgs a2 = a;  // a balanced plan launches only the segments g >= 1, longest first
         a2.order = order2;

@@ -12,8 +12,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <utility>
-
 #include "../../include/kda.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -215,33 +213,6 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 template <typename Kern>
 inline bool set_smem_attr(Kern kern, uint32_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) == cudaSuccess;
-}
-
-// Programmatic dependent launch: a kernel launched by launch_dependent may start
-// (be scheduled, run its prologue) while the kernel before it in the stream is
-// still running.  It must call pdl_wait() before it reads anything that kernel
-// writes: the wait returns once the previous grid has completed and its writes are
-// visible (at once when the kernel was launched without the attribute).  A kernel
-// calls pdl_trigger() to let the next one launch early; the next grid then starts
-// only after every CTA of this one has triggered or exited, so the two cannot
-// deadlock over SM resources.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                                    Args&&... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // Two fp32 -> packed bf16x2, rounding to nearest on the bit pattern (ties away
