@@ -191,6 +191,18 @@ def test_balanced_plan_with_empty_sequences_and_no_initial_state(kda):
     assert eo < TOL and es < TOL, (eo, es)
 
 
+def test_balanced_plan_fp32_inputs_with_l2norm(kda):
+    """fp32 q, k, v (rounded to bf16 operands, fp32 o) normalised in the kernel, on a
+    packed call the device plan cuts (one 38-chunk sequence among short ones)."""
+    cu = [0, 100, 2500, 2600, 2700, 2701, 2800, 2900, 3000]
+    assert kda.chunk_fwd_segments(1, cu[-1], 16, len(cu) - 1) == (-1, -1)
+    inp = synth.op_inputs(B=len(cu) - 1, H=16, T=cu[-1], dtype=torch.float32, s0_std=0.02, seed=34, cu_seqlens=cu)
+    inp["q"] = inp["q"] * 3.0
+    inp["k"] = inp["k"] * 0.5
+    eo, es = run_both(kda, inp, l2=True, heads=[2, 9])
+    assert eo < TOL and es < TOL, (eo, es)
+
+
 def test_final_state_only_and_zero_state(kda):
     inp = synth.op_inputs(B=2, H=2, T=100, s0_std=None, seed=14)
     eo, es = run_both(kda, inp)

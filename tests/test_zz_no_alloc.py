@@ -33,16 +33,25 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("case", ["dense_4k_scan", "varlen"])
+@pytest.mark.parametrize("case", ["dense_4k_scan", "varlen", "varlen_balanced"])
 def test_noalloc_matches_workspace_entry_point_two_calls(kda, case):
+    """varlen_balanced: 8 packed sequences x 8 heads, one of them 38 chunks long, so the
+    device plan cuts it; the full workspace (product images and per-segment states,
+    ~50 MB) fits the static array, so both entry points run the same cuts."""
     fn = _noalloc(kda)
     dev = torch.device("cuda")
     if case == "dense_4k_scan":
         inp = synth.op_inputs(**synth.PREFILL_4K, device=dev)
         cu = None
-    else:
+    elif case == "varlen":
         cuv = [0, 5, 69, 70, 300, 777]
         inp = synth.op_inputs(B=len(cuv) - 1, H=3, T=cuv[-1], s0_std=0.02, seed=31, cu_seqlens=cuv, device=dev)
+        cu = inp["cu_seqlens"]
+    else:
+        cuv = [0, 100, 2500, 2600, 2700, 2701, 2800, 2900, 3000]
+        assert kda.chunk_fwd_segments(1, cuv[-1], 8, len(cuv) - 1) == (-1, -1)
+        assert kda.chunk_fwd_workspace_bytes(1, cuv[-1], 8, len(cuv) - 1) <= 64 << 20
+        inp = synth.op_inputs(B=len(cuv) - 1, H=8, T=cuv[-1], s0_std=0.02, seed=35, cu_seqlens=cuv, device=dev)
         cu = inp["cu_seqlens"]
     q, k, v, g, beta, s0 = (inp[n] for n in ("q", "k", "v", "g", "beta", "s0"))
     B, T, H, _ = q.shape
