@@ -207,6 +207,63 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;  // exp(x) = 2^(x log2 e)
 
+// ---- exact A and P for a chunk whose decay range fails the factored path's bound:
+// one exp per (r, i, c) term with every exponent <= 0, one (r, i) pair of the 64 x 65 / 2
+// lower-triangle pairs per thread and step (kThreads = 512 threads)
+constexpr int kExactPairs = 64 * 65 / 2, kExactPer = (kExactPairs + 511) / 512;
+struct ExactAP {
+    float ra[kExactPer], rp[kExactPer];  // the thread's A and P terms
+};
+__device__ __forceinline__ void exact_pair(int pidx, int& r, int& i) {  // pidx = r (r + 1) / 2 + i, i <= r
+    r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
+    while (r * (r + 1) / 2 > pidx) --r;
+    while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
+    i = pidx - r * (r + 1) / 2;
+}
+
+
+// The terms, from the q, k and cumulative-gate tiles (rows >= len are zero).
+__device__ __noinline__ void exact_ap_terms(const uint8_t* sm, int tid, int len, ExactAP* acc) {
+    const float* sB = reinterpret_cast<const float*>(sm + OFF_G);
+    const uint8_t* sQb = sm + OFF_Q;
+    const uint8_t* sKb = sm + OFF_K;
+    for (int u = 0; u < kExactPer; ++u) {
+        const int pidx = tid + u * 512;
+        acc->ra[u] = acc->rp[u] = 0.f;
+        if (pidx >= kExactPairs) continue;
+        int r, i;
+        exact_pair(pidx, r, i);
+        if (r < len) {
+            float ra = 0.f, rp = 0.f;
+            for (int cc = 0; cc < kD; ++cc) {
+                const float f = __expf(sB[r * kD + cc] - sB[i * kD + cc]);
+                const uint32_t offr = uint32_t(cc >> 6) * 8192u + sw128_off(r, cc & 63);
+                const uint32_t offi = uint32_t(cc >> 6) * 8192u + sw128_off(i, cc & 63);
+                const float ki = bf16_at(sKb, offi) * f;
+                ra += bf16_at(sKb, offr) * ki;
+                rp += bf16_at(sQb, offr) * ki;
+            }
+            acc->ra[u] = ra;
+            acc->rp[u] = rp;
+        }
+    }
+}
+// A (beta-scaled, strictly lower; diagonal blocks transposed for the UT solve) into sA and
+// P (bf16, lower incl. the diagonal, times scale) into its tile; every thread of the CTA calls it.
+__device__ __noinline__ void exact_ap_store(uint8_t* sm, uint32_t sbase, float* sA, const float* sBeta, float scale,
+                                            int tid, const ExactAP* acc) {
+    for (int e = tid; e < 64 * 64; e += 512) sA[e] = 0.f;
+    for (int e = tid; e < 512; e += 512) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int u = 0; u < kExactPer; ++u) {
+        const int pidx = tid + u * 512;
+        if (pidx >= kExactPairs) continue;
+        int r, i;
+        exact_pair(pidx, r, i);
+        if (i < r) sA[((r >> 4) == (i >> 4)) ? sidx(i, r) : sidx(r, i)] = sBeta[r] * acc->ra[u];
+        *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) = __float2bfloat16_rn(acc->rp[u] * scale);
+    }
+}
 
 // kSummary = true : segment summary (zero start state, identity X, no output).
 // kSummary = false: output from the segment's true start state (the initial state
@@ -711,50 +768,15 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap& tm_q, const CUtens
                 }
             }
         } else {
-            // Exact fallback: one exp per (r, i, c) term, all exponents <= 0.
-            const float* sB = reinterpret_cast<const float*>(sm + OFF_G);
-            const uint8_t* sQb = sm + OFF_Q;
-            const uint8_t* sKb = sm + OFF_K;
-            constexpr int kPairs = 64 * 65 / 2, kPer = (kPairs + kThreads - 1) / kThreads;
-            float ra[kPer], rp[kPer];
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                const int pidx = tid + u * kThreads;
-                ra[u] = rp[u] = 0.f;
-                if (pidx >= kPairs) continue;
-                int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
-                while (r * (r + 1) / 2 > pidx) --r;
-                while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
-                const int i = pidx - r * (r + 1) / 2;
-                if (r < len) {
-                    for (int cc = 0; cc < kD; ++cc) {
-                        const float f = __expf(sB[r * kD + cc] - sB[i * kD + cc]);
-                        const uint32_t offr = uint32_t(cc >> 6) * 8192u + sw128_off(r, cc & 63);
-                        const uint32_t offi = uint32_t(cc >> 6) * 8192u + sw128_off(i, cc & 63);
-                        const float ki = bf16_at(sKb, offi) * f;
-                        ra[u] += bf16_at(sKb, offr) * ki;
-                        rp[u] += bf16_at(sQb, offr) * ki;
-                    }
-                }
-            }
+            // Exact fallback: one exp per (r, i, c) term, all exponents <= 0.  Out of line: it is
+            // rare, and inline it would sit in the middle of the chunk loop's instruction stream.
+            ExactAP ex;
+            exact_ap_terms(sm, tid, len, &ex);
             __syncthreads();  // the q / k / b tiles are read
             if (tid == kLoader && c + 1 < nchunks) {
                 pend_qkg = issue_qkg(c + 1);
             }
-            for (int e = tid; e < 64 * 64; e += kThreads) sA[e] = 0.f;
-            for (int e = tid; e < 512; e += kThreads) st_shared_v4(sbase + OFF_P + e * 16, 0u, 0u, 0u, 0u);
-            __syncthreads();
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                const int pidx = tid + u * kThreads;
-                if (pidx >= kPairs) continue;
-                int r = int((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
-                while (r * (r + 1) / 2 > pidx) --r;
-                while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
-                const int i = pidx - r * (r + 1) / 2;
-                if (i < r) sA[((r >> 4) == (i >> 4)) ? sidx(i, r) : sidx(r, i)] = sBeta[r] * ra[u];
-                *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw128_off(r, i)) = __float2bfloat16_rn(rp[u] * p.scale);
-            }
+            exact_ap_store(sm, sbase, sA, sBeta, p.scale, tid, &ex);
         }
         KDA_WMARK(0);
         tc_fence_before();
