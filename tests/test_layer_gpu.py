@@ -8,8 +8,8 @@ The per-(token, head) RMSNorm carries each row's relative error into y at full
 weight, and for rows whose RMS is far below the norm's epsilon (the first
 tokens of a sequence, o ~ beta (k.q) v) absolute errors pass straight through,
 so the shortest sequences sit closest to the bar (about 9e-3 for 4 tokens).
-Tolerance: relative L2 <= 1e-2 on y and on the final state (the benchmark spec's
-bar for outputs and states)."""
+Tolerance: relative L2 <= 1e-2 on y and on the final state (the bar the
+operator's outputs and states are held to)."""
 import numpy as np
 import pytest
 import torch
