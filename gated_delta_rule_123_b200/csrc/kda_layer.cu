@@ -54,8 +54,10 @@ __device__ __forceinline__ int seq_begin(const int32_t* cu, int seq_len, int n) 
 // cached history conv_in [nseq][3][3 H 128] (row 2 = the token just before) or
 // from zero.  Loads and stores are 16 bytes, and all of a block's rows are
 // requested before the first is used (the kernel is bound by memory latency
-// otherwise).
-constexpr int kConvTok = 8;
+// otherwise).  Each block also re-reads the three rows before it: 12 tokens per
+// block read 15/12 of the rows (8 tokens: 11/8) and still fit 128 registers
+// (16 tokens spill).
+constexpr int kConvTok = 12;
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
