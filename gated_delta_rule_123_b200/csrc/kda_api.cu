@@ -109,6 +109,7 @@ int kda_chunk_fwd_segment_tokens(int B, int T, int H, int num_seqs, int* middle_
 
 int kda_chunk_fwd_plan_items(const void* workspace, int B, int T, int H, int num_seqs, int* rows, int max_rows) {
     if (!workspace || !rows || max_rows < 0 || B < 0 || T < 0 || H < 0 || num_seqs < 0) return -1;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;  // the call may have run on any stream
     return chunk_plan_items(workspace, B, T, H, num_seqs, rows, max_rows);
 }
 
