@@ -28,6 +28,9 @@ Parts:
 * ``kda_layer``               the full KDA layer (numpy + the recurrence).
 * ``kda_recurrent_backward``  reverse mode of the recurrence (numpy): dq, dk, dv,
                               dg, dbeta and the initial-state gradient.
+* ``kda_chunkwise_backward`` reverse mode of the chunkwise form (numpy), chunk by
+                              chunk: the same six gradients through the gated grams,
+                              the WY products and the UT inverse.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against facts the
 pages and plain mathematics fix (special cases, closed forms, invariants, an
@@ -43,6 +46,7 @@ import numpy as np
 
 from .backward import kda_recurrent_backward  # noqa: F401
 from .chunkwise import kda_chunkwise  # noqa: F401
+from .chunkwise_backward import kda_chunkwise_backward  # noqa: F401
 from .layer import kda_layer, layer_reference_parts  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

@@ -91,3 +91,25 @@ def test_backward_batched_heads_match_single():
                                                 s0=s0[b, h], ds_final=dsT[b, h])
             assert np.allclose(full[0][b, :, h], one[0][:, 0]) and np.allclose(full[3][b, :, h], one[3][:, 0])
             assert np.allclose(full[4][b, :, h], one[4][:, 0]) and np.allclose(full[5][b, h], one[5][0, 0])
+
+
+def test_chunkwise_backward_equals_recurrent_backward():
+    """The chunk-form reverse mode (written from the chunkwise forward, line by line)
+    against the token-by-token reverse mode pinned above: chunk sizes from 1 to 64,
+    ragged last chunks, strong decay, a q scale, several sequences and heads."""
+    cases = ((1, 7, 1, 5, 3, 0.3, 1.0), (2, 40, 2, 6, 16, 0.3, 0.7), (1, 33, 1, 4, 64, 2.0, 1.0),
+             (1, 10, 1, 3, 1, 0.3, 1.3), (1, 70, 1, 8, 64, 0.3, 1.0))
+    for B, T, H, D, C, gate, scale in cases:
+        r = np.random.default_rng(B * 1000 + T)
+        unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)  # noqa: E731
+        q, k = unit(r.standard_normal((B, T, H, D))), unit(r.standard_normal((B, T, H, D)))
+        v = r.standard_normal((B, T, H, D))
+        g = -gate * np.log1p(np.exp(r.standard_normal((B, T, H, D))))
+        beta = 1 / (1 + np.exp(-r.standard_normal((B, T, H))))
+        s0, do, ds = 0.3 * r.standard_normal((B, H, D, D)), r.standard_normal((B, T, H, D)), r.standard_normal((B, H, D, D))
+        a = oracle.kda_chunkwise_backward(q, k, v, g, beta, do, s0=s0, ds_final=ds, scale=scale, chunk=C)
+        b = oracle.kda_recurrent_backward(q, k, v, g, beta, do, s0=s0, ds_final=ds, scale=scale)
+        for name, x, y in zip(("dq", "dk", "dv", "dg", "dbeta", "ds0"), a, b):
+            err = np.max(np.abs(x - y)) / np.max(np.abs(y))
+            assert err < 1e-12, (B, T, H, D, C, name, err)
+
